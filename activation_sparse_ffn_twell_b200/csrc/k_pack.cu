@@ -1,0 +1,205 @@
+// TwELL packing of a dense bf16 hidden matrix, and the overflow finaliser that
+// turns the unordered staged backup into the canonical ascending list.
+//
+// TwELL (upppp.jp 2026-05-11, section 「TwELLとカスタムCUDAカーネルが解決する課題」):
+// hidden columns are cut into tiles of tile_w; per (token, tile) the nonzeros are
+// kept as ELL slots (value, in-tile index) in ascending column order; a pair with
+// more than ell_w nonzeros also keeps its dense segment in the backup.
+//
+// Packing is HBM-bound (read h once, write the packed form once): one warp per
+// (token, tile) pair, lanes own contiguous column groups so the read is a single
+// coalesced segment, and slot positions come from warp ballots + popcounts.
+#include "twell_device.cuh"
+
+namespace twell {
+namespace {
+
+template <int TW>
+__global__ void __launch_bounds__(256) k_pack_dense(const uint16_t *__restrict__ h, int ld_h,
+                                                    PackTarget p) {
+  constexpr int EPL = TW / 32;  // elements per lane (1, 2, 4, 8)
+  const int lane = threadIdx.x & 31;
+  const int warps_per_cta = blockDim.x >> 5;
+  const long long n_pairs = static_cast<long long>(p.M) * p.T;
+  const unsigned full = 0xFFFFFFFFu;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  for (long long pair = static_cast<long long>(blockIdx.x) * warps_per_cta + (threadIdx.x >> 5);
+       pair < n_pairs; pair += static_cast<long long>(gridDim.x) * warps_per_cta) {
+    const int r = static_cast<int>(pair / p.T);
+    const int t = static_cast<int>(pair - static_cast<long long>(r) * p.T);
+    const uint16_t *src = h + static_cast<size_t>(r) * ld_h + static_cast<size_t>(t) * TW + lane * EPL;
+
+    uint16_t v[EPL];
+    if constexpr (EPL == 8) {
+      uint4 q = __ldg(reinterpret_cast<const uint4 *>(src));
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { v[2 * i] = w[i] & 0xFFFF; v[2 * i + 1] = w[i] >> 16; }
+    } else if constexpr (EPL == 4) {
+      uint2 q = __ldg(reinterpret_cast<const uint2 *>(src));
+      v[0] = q.x & 0xFFFF; v[1] = q.x >> 16; v[2] = q.y & 0xFFFF; v[3] = q.y >> 16;
+    } else if constexpr (EPL == 2) {
+      uint32_t q = __ldg(reinterpret_cast<const unsigned int *>(src));
+      v[0] = q & 0xFFFF; v[1] = q >> 16;
+    } else {
+      v[0] = __ldg(src);
+    }
+
+    // rank of each nonzero among the pair's nonzeros in ascending column order
+    int before = 0;   // nonzeros in lanes below this one
+    int total = 0;
+    unsigned nzbits = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const bool nz = (v[i] & 0x7FFF) != 0;
+      nzbits |= (nz ? 1u : 0u) << i;
+      const unsigned m = __ballot_sync(full, nz);
+      before += __popc(m & lt_mask);
+      total += __popc(m);
+    }
+    const size_t rec = static_cast<size_t>(pair) * p.E;
+    int rank = before;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      if ((nzbits >> i) & 1u) {
+        if (rank < p.E) {
+          p.vals[rec + rank] = v[i];
+          p.idx[rec + rank] = static_cast<uint8_t>(lane * EPL + i);
+        }
+        ++rank;
+      }
+    }
+    for (int s = total + lane; s < p.E; s += 32) {   // padding slots: (+0, 0)
+      p.vals[rec + s] = 0;
+      p.idx[rec + s] = 0;
+    }
+    if (lane == 0) p.nnz[pair] = static_cast<uint16_t>(total);
+
+    if (total > p.E) {   // warp-uniform: stage the dense segment
+      int k = 0;
+      if (lane == 0) {
+        k = atomicAdd(p.stage_ctr, 1);
+        atomicAdd(p.row_ovf + r, 1);
+        if (k < p.cap) p.stage_pos[k] = static_cast<int32_t>(pair);
+      }
+      k = __shfl_sync(full, k, 0);
+      if (k < p.cap) {
+        uint16_t *dst = p.stage_dense + static_cast<size_t>(k) * TW + lane * EPL;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) dst[i] = ((v[i] & 0x7FFF) != 0) ? v[i] : 0;
+      }
+    }
+  }
+}
+
+// Exclusive scan of the per-token overflow counts (one CTA, any M), total ->
+// n_ovf, capacity check -> status.
+__global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
+  __shared__ int warp_sums[32];
+  __shared__ int carry_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) carry_s = 0;
+  __syncthreads();
+  for (int base = 0; base < p.M; base += 1024) {
+    const int i = base + tid;
+    const int v = (i < p.M) ? p.row_ovf[i] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int ws = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xFFFFFFFFu, ws, o);
+        if (lane >= o) ws += n;
+      }
+      warp_sums[lane] = ws;   // inclusive over warps
+    }
+    __syncthreads();
+    const int carry = carry_s;
+    const int excl = carry + (warp ? warp_sums[warp - 1] : 0) + incl - v;
+    if (i < p.M) p.row_prefix[i] = excl;
+    __syncthreads();
+    if (tid == 1023) carry_s = carry + warp_sums[31];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    *p.n_ovf = carry_s;
+    if (carry_s > p.cap) raise_status(p.status, TWELL_ERR_OVERFLOW_CAPACITY);
+  }
+}
+
+// Move each staged segment to its rank in the ascending r*T+t order.
+template <int TW>
+__global__ void __launch_bounds__(256) k_ovf_scatter(PackTarget p) {
+  const int lane = threadIdx.x & 31;
+  const int warps_per_cta = blockDim.x >> 5;
+  const int staged = min(*p.stage_ctr, p.cap);
+  for (int k = blockIdx.x * warps_per_cta + (threadIdx.x >> 5); k < staged;
+       k += gridDim.x * warps_per_cta) {
+    const int pos = p.stage_pos[k];
+    const int r = pos / p.T, t = pos - r * p.T;
+    int before = 0;
+    for (int t0 = 0; t0 < t; t0 += 32) {
+      const int tt = t0 + lane;
+      const bool ov = (tt < t) && (static_cast<int>(p.nnz[static_cast<size_t>(r) * p.T + tt]) > p.E);
+      before += __popc(__ballot_sync(0xFFFFFFFFu, ov));
+    }
+    const int rank = p.row_prefix[r] + before;
+    if (rank >= p.cap) continue;
+    if (lane == 0) p.ovf_pos[rank] = pos;
+    const uint16_t *src = p.stage_dense + static_cast<size_t>(k) * TW;
+    uint16_t *dst = p.ovf_dense + static_cast<size_t>(rank) * TW;
+    constexpr int kVec = TW / 8;   // 16-byte vectors per segment (4 .. 32)
+    for (int c = lane; c < kVec; c += 32)
+      reinterpret_cast<uint4 *>(dst)[c] = reinterpret_cast<const uint4 *>(src)[c];
+  }
+}
+
+int grid_for(long long work_items, int per_cta, int cap_ctas) {
+  long long g = (work_items + per_cta - 1) / per_cta;
+  if (g < 1) g = 1;
+  if (g > cap_ctas) g = cap_ctas;
+  return static_cast<int>(g);
+}
+
+}  // namespace
+
+cudaError_t launch_pack_dense(const uint16_t *h, int ld_h, const PackTarget &t, cudaStream_t s) {
+  const long long pairs = static_cast<long long>(t.M) * t.T;
+  if (pairs == 0) return cudaSuccess;
+  const int grid = grid_for(pairs, 8, 148 * 64);
+  switch (t.tw) {
+    case 32: k_pack_dense<32><<<grid, 256, 0, s>>>(h, ld_h, t); break;
+    case 64: k_pack_dense<64><<<grid, 256, 0, s>>>(h, ld_h, t); break;
+    case 128: k_pack_dense<128><<<grid, 256, 0, s>>>(h, ld_h, t); break;
+    case 256: k_pack_dense<256><<<grid, 256, 0, s>>>(h, ld_h, t); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {
+  if (t.M == 0) return cudaSuccess;
+  k_ovf_row_scan<<<1, 1024, 0, s>>>(t);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (t.cap == 0) return cudaSuccess;
+  const int grid = grid_for(t.cap, 8, 148 * 8);
+  switch (t.tw) {
+    case 32: k_ovf_scatter<32><<<grid, 256, 0, s>>>(t); break;
+    case 64: k_ovf_scatter<64><<<grid, 256, 0, s>>>(t); break;
+    case 128: k_ovf_scatter<128><<<grid, 256, 0, s>>>(t); break;
+    case 256: k_ovf_scatter<256><<<grid, 256, 0, s>>>(t); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace twell

@@ -1,0 +1,306 @@
+// Host side of the C ABI declared in include/twell.h: argument validation,
+// workspace carve-up, tensor-map encoding and kernel launch order.  Nothing here
+// computes on the host; every step of the layer runs in the kernels.
+#include <cstring>
+#include <mutex>
+
+#include "twell_internal.h"
+
+namespace twell {
+
+cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s);
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_tile(int tile_w) { return tile_w == 32 || tile_w == 64 || tile_w == 128 || tile_w == 256; }
+
+// Shape rules shared by every call.
+twell_status check_shape(int M, int d_ff, int tile_w, int ell_w) {
+  if (M < 0 || d_ff <= 0 || !valid_tile(tile_w) || d_ff % tile_w != 0) return TWELL_ERR_INVALID_ARG;
+  if (ell_w < 1 || ell_w > tile_w) return TWELL_ERR_INVALID_ARG;
+  return TWELL_OK;
+}
+
+twell_status check_matrix(const twell_matrix *a, int M, int d_ff, int tile_w, int ell_w) {
+  if (a == nullptr) return TWELL_ERR_INVALID_ARG;
+  if (a->M != M || a->d_ff != d_ff || a->tile_w != tile_w || a->ell_w != ell_w)
+    return TWELL_ERR_INVALID_ARG;
+  if (a->ovf_capacity < 0 || a->n_ovf == nullptr || a->status == nullptr) return TWELL_ERR_INVALID_ARG;
+  if (M > 0 && (a->vals == nullptr || a->idx == nullptr || a->nnz == nullptr)) return TWELL_ERR_INVALID_ARG;
+  if (!a16(a->vals) || !a16(a->idx) || !a16(a->nnz)) return TWELL_ERR_INVALID_ARG;
+  if (a->ovf_capacity > 0 && (a->ovf_pos == nullptr || a->ovf_dense == nullptr)) return TWELL_ERR_INVALID_ARG;
+  if (!a16(a->ovf_pos) || !a16(a->ovf_dense)) return TWELL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a->n_ovf) & 3u) || (reinterpret_cast<uintptr_t>(a->status) & 3u))
+    return TWELL_ERR_INVALID_ARG;
+  return TWELL_OK;
+}
+
+// Workspace regions: overflow staging + per-block path flags.
+struct Ws {
+  WsLayout L;
+  size_t blk_path;
+  size_t total;
+};
+
+Ws ws_plan(int M, int tile_w, int cap) {
+  Ws w;
+  w.L = ws_layout(M, tile_w, cap);
+  w.blk_path = w.L.total;
+  w.total = align256(w.blk_path + sizeof(int32_t) * static_cast<size_t>((M + kBlockM - 1) / kBlockM + 1));
+  return w;
+}
+
+PackTarget make_target(const twell_matrix *a, void *ws) {
+  const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  PackTarget t;
+  t.M = a->M; t.f = a->d_ff; t.tw = a->tile_w; t.E = a->ell_w; t.T = a->d_ff / a->tile_w;
+  t.vals = a->vals; t.idx = a->idx; t.nnz = a->nnz;
+  t.cap = a->ovf_capacity; t.n_ovf = a->n_ovf; t.ovf_pos = a->ovf_pos; t.ovf_dense = a->ovf_dense;
+  t.status = a->status;
+  t.stage_ctr = reinterpret_cast<int32_t *>(base + w.L.ctr);
+  t.row_ovf = reinterpret_cast<int32_t *>(base + w.L.row_ovf);
+  t.row_prefix = reinterpret_cast<int32_t *>(base + w.L.row_prefix);
+  t.stage_pos = reinterpret_cast<int32_t *>(base + w.L.stage_pos);
+  t.stage_dense = reinterpret_cast<uint16_t *>(base + w.L.stage_dense);
+  return t;
+}
+
+TwellView make_view(const twell_matrix *a) {
+  TwellView v;
+  v.M = a->M; v.f = a->d_ff; v.tw = a->tile_w; v.E = a->ell_w; v.T = a->d_ff / a->tile_w;
+  v.vals = a->vals; v.idx = a->idx; v.nnz = a->nnz;
+  v.cap = a->ovf_capacity; v.n_ovf = a->n_ovf; v.ovf_pos = a->ovf_pos; v.ovf_dense = a->ovf_dense;
+  v.status = a->status;
+  return v;
+}
+
+twell_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TWELL_OK : TWELL_ERR_CUDA; }
+
+// Reset the status word and the overflow staging counters before a producer runs.
+twell_status reset_for_pack(const PackTarget &t, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(t.status, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  const size_t bytes = reinterpret_cast<uint8_t *>(t.row_ovf + t.M) - reinterpret_cast<uint8_t *>(t.stage_ctr);
+  e = cudaMemsetAsync(t.stage_ctr, 0, bytes, s);
+  return from_cuda(e);
+}
+
+twell_status check_ws(void *ws, size_t ws_bytes, int M, int tile_w, int cap) {
+  const Ws w = ws_plan(M, tile_w, cap);
+  if (ws == nullptr || !a16(ws) || ws_bytes < w.total) return TWELL_ERR_WORKSPACE;
+  return TWELL_OK;
+}
+
+twell_status up_pack_checked(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                             const uint16_t *b, int M, int d_model, int d_ff, int tile_w, int ell_w,
+                             const twell_matrix *out, float *z_debug, void *ws, size_t ws_bytes,
+                             cudaStream_t s) {
+  if (M == 0) return TWELL_OK;
+  const PackTarget t = make_target(out, ws);
+  const int sms = sm_count();
+  if (sms <= 0) return TWELL_ERR_CUDA;
+  twell_status st = reset_for_pack(t, s);
+  if (st != TWELL_OK) return st;
+  UpArgs a;
+  a.x = x; a.w_up = W_up; a.w_gate = W_gate; a.b = b;
+  a.M = M; a.d = d_model; a.f = d_ff; a.z_debug = z_debug;
+  cudaError_t e = launch_up_pack(a, t, sms, s);
+  if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  return from_cuda(launch_overflow_finalize(t, s));
+}
+
+twell_status validate_up(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                         const uint16_t *b, int M, int d_model, int d_ff, int tile_w, int ell_w,
+                         const twell_matrix *out, float *z_debug, void *ws, size_t ws_bytes) {
+  twell_status st = check_shape(M, d_ff, tile_w, ell_w);
+  if (st != TWELL_OK) return st;
+  if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
+  if (M == 0) return TWELL_OK;   // documented no-op
+  if (x == nullptr || W_up == nullptr || !a16(x) || !a16(W_up) || !a16(W_gate) || !a16(b) ||
+      !a16(z_debug))
+    return TWELL_ERR_INVALID_ARG;
+  st = check_matrix(out, M, d_ff, tile_w, ell_w);
+  if (st != TWELL_OK) return st;
+  if (ell_w > kMaxEllFused) return TWELL_ERR_UNSUPPORTED;
+  if (W_gate != nullptr && tile_w > 128) return TWELL_ERR_UNSUPPORTED;
+  return check_ws(ws, ws_bytes, M, tile_w, out->ovf_capacity);
+}
+
+twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
+                           int mode, void *ws, size_t ws_bytes) {
+  if (a == nullptr) return TWELL_ERR_INVALID_ARG;
+  twell_status st = check_shape(a->M, a->d_ff, a->tile_w, a->ell_w);
+  if (st != TWELL_OK) return st;
+  if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
+  if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
+    return TWELL_ERR_INVALID_ARG;
+  if (a->M == 0) return TWELL_OK;   // documented no-op
+  st = check_matrix(a, a->M, a->d_ff, a->tile_w, a->ell_w);
+  if (st != TWELL_OK) return st;
+  if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
+  if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y)) return TWELL_ERR_INVALID_ARG;
+  if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
+    return TWELL_ERR_INVALID_ARG;
+  return check_ws(ws, ws_bytes, a->M, a->tile_w, a->ovf_capacity);
+}
+
+twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
+                          int mode, void *ws, cudaStream_t s) {
+  if (a->M == 0) return TWELL_OK;
+  const TwellView v = make_view(a);
+  const int sms = sm_count();
+  if (sms <= 0) return TWELL_ERR_CUDA;
+  if (mode == TWELL_DOWN_GATHER) return from_cuda(launch_spmm_gather(v, W_down, d_model, y, nullptr, s));
+  if (mode == TWELL_DOWN_MMA) return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, s));
+  const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
+  int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
+  cudaError_t e = launch_block_path(v, kDownCrossoverDensity, blk, s);
+  if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  e = launch_spmm_gather(v, W_down, d_model, y, blk, s);
+  if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sms, s));
+}
+
+}  // namespace
+
+CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                              uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t elem_strides[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace twell
+
+using namespace twell;
+
+extern "C" {
+
+int twell_version(void) { return 100; }
+
+const char *twell_status_string(twell_status s) {
+  switch (s) {
+    case TWELL_OK: return "ok";
+    case TWELL_ERR_INVALID_ARG: return "invalid argument";
+    case TWELL_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TWELL_ERR_OVERFLOW_CAPACITY: return "overflow backup capacity exhausted";
+    case TWELL_ERR_CUDA: return "CUDA error";
+    case TWELL_ERR_TIMEOUT: return "device wait timed out";
+    case TWELL_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w, int gated,
+                             int ovf_capacity) {
+  if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0) return 0;
+  if (d_model <= 0 || d_model % 64 != 0 || (gated != 0 && gated != 1)) return 0;
+  return ws_plan(M, tile_w, ovf_capacity).total;
+}
+
+twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
+                        const twell_matrix *out, void *ws, size_t ws_bytes, void *stream) {
+  twell_status st = check_shape(M, d_ff, tile_w, ell_w);
+  if (st != TWELL_OK) return st;
+  if (M == 0) return TWELL_OK;   // documented no-op: nothing is read or written
+  if (h == nullptr || !a16(h) || ld_h < d_ff || ld_h % 8 != 0) return TWELL_ERR_INVALID_ARG;
+  st = check_matrix(out, M, d_ff, tile_w, ell_w);
+  if (st != TWELL_OK) return st;
+  st = check_ws(ws, ws_bytes, M, tile_w, out->ovf_capacity);
+  if (st != TWELL_OK) return st;
+  if (M == 0) return TWELL_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const PackTarget t = make_target(out, ws);
+  st = reset_for_pack(t, s);
+  if (st != TWELL_OK) return st;
+  if (launch_pack_dense(h, ld_h, t, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  return from_cuda(launch_overflow_finalize(t, s));
+}
+
+twell_status twell_up_pack(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                           const uint16_t *b, int M, int d_model, int d_ff, int tile_w, int ell_w,
+                           const twell_matrix *out, float *z_debug, void *ws, size_t ws_bytes,
+                           void *stream) {
+  twell_status st = validate_up(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, out, z_debug,
+                                ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  return up_pack_checked(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, out, z_debug, ws,
+                         ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+twell_status twell_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
+                        int mode, void *ws, size_t ws_bytes, void *stream) {
+  twell_status st = validate_spmm(a, W_down, d_model, y, mode, ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  return spmm_checked(a, W_down, d_model, y, mode, ws, static_cast<cudaStream_t>(stream));
+}
+
+twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                               const uint16_t *b, const uint16_t *W_down, int M, int d_model,
+                               int d_ff, int tile_w, int ell_w, const twell_matrix *twell, uint16_t *y,
+                               int mode, void *ws, size_t ws_bytes, void *stream) {
+  twell_status st = validate_up(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, twell, nullptr,
+                                ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  st = validate_spmm(twell, W_down, d_model, y, mode, ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = up_pack_checked(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, twell, nullptr, ws,
+                       ws_bytes, s);
+  if (st != TWELL_OK) return st;
+  return spmm_checked(twell, W_down, d_model, y, mode, ws, s);
+}
+
+twell_status twell_read_status(const twell_matrix *a, void *stream, int32_t *n_ovf_out) {
+  if (a == nullptr || a->status == nullptr || a->n_ovf == nullptr) return TWELL_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TWELL_ERR_CUDA;
+  int32_t st = 0, n = 0;
+  if (cudaMemcpy(&st, a->status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return TWELL_ERR_CUDA;
+  if (cudaMemcpy(&n, a->n_ovf, sizeof(n), cudaMemcpyDeviceToHost) != cudaSuccess) return TWELL_ERR_CUDA;
+  if (n_ovf_out) *n_ovf_out = n;
+  return static_cast<twell_status>(st);
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// Internal definitions shared by the host-side API and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/twell.h"
+
+namespace twell {
+
+// Bounded device waits: give up after ~2 s of wall time (a healthy wait in these
+// kernels lasts microseconds) or this many polls, whichever comes first.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr uint32_t kWaitMaxIters = 1u << 30;
+
+// Tile shapes of the tensor-core kernels.
+constexpr int kBlockM = 128;   // tokens per accumulator tile (TMEM lanes)
+constexpr int kBlockK = 64;    // K elements per pipeline stage (one 128-byte swizzle row)
+constexpr int kUmmaK = 16;     // K per tcgen05.mma (bf16)
+constexpr int kMaxEllFused = 64;
+
+// Device view of a TwELL matrix plus the overflow staging area in the workspace.
+struct PackTarget {
+  int M, f, tw, E, T;
+  uint16_t *vals;
+  uint8_t *idx;
+  uint16_t *nnz;
+  int cap;
+  int32_t *n_ovf;
+  int32_t *ovf_pos;
+  uint16_t *ovf_dense;
+  int32_t *status;
+  // workspace
+  int32_t *stage_ctr;      // [1] number of staged overflow segments (unsorted)
+  int32_t *row_ovf;        // [M] overflow pairs per token
+  int32_t *row_prefix;     // [M] exclusive prefix of row_ovf
+  int32_t *stage_pos;      // [cap] r*T+t of each staged segment
+  uint16_t *stage_dense;   // [cap][tw] staged dense segments
+};
+
+// Read-only device view used by the down-projection kernels.
+struct TwellView {
+  int M, f, tw, E, T;
+  const uint16_t *vals;
+  const uint8_t *idx;
+  const uint16_t *nnz;
+  int cap;
+  const int32_t *n_ovf;
+  const int32_t *ovf_pos;
+  const uint16_t *ovf_dense;
+  int32_t *status;
+};
+
+// Workspace carve-up (every region 256-byte aligned).
+struct WsLayout {
+  size_t ctr, row_ovf, row_prefix, stage_pos, stage_dense, total;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+inline WsLayout ws_layout(int M, int tile_w, int cap) {
+  WsLayout L;
+  size_t o = 0;
+  L.ctr = o;         o = align256(o + 64);
+  L.row_ovf = o;     o = align256(o + sizeof(int32_t) * static_cast<size_t>(M));
+  L.row_prefix = o;  o = align256(o + sizeof(int32_t) * static_cast<size_t>(M));
+  L.stage_pos = o;   o = align256(o + sizeof(int32_t) * static_cast<size_t>(cap));
+  L.stage_dense = o; o = align256(o + 2 * static_cast<size_t>(cap) * tile_w);
+  L.total = o;
+  return L;
+}
+
+// ---------------------------------------------------------------------------
+// Launchers (defined next to their kernels).  Each returns cudaSuccess or the
+// launch error; none synchronises.
+// ---------------------------------------------------------------------------
+cudaError_t launch_pack_dense(const uint16_t *h, int ld_h, const PackTarget &t, cudaStream_t s);
+cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s);
+
+struct UpArgs {
+  const uint16_t *x, *w_up, *w_gate, *b;
+  int M, d, f;
+  float *z_debug;
+};
+cudaError_t launch_up_pack(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
+
+// blk_path: NULL (the kernel owns every token block) or one int per 128-token
+// block: 0 = gather path owns it, 1 = tensor-core path owns it.
+cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
+                               const int32_t *blk_path, cudaStream_t s);
+cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
+                            const int32_t *blk_path, int num_sms, cudaStream_t s);
+
+// Density (nonzeros / (rows * d_ff)) of a 128-token block at or above which the
+// AUTO down-projection uses the tensor-core path.  Chosen from measurement.
+constexpr float kDownCrossoverDensity = 0.02f;
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved at run time so the
+// library loads on machines without a driver).
+CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                              uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                              CUtensorMapSwizzle swizzle);
+
+}  // namespace twell

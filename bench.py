@@ -1,0 +1,483 @@
+#!/usr/bin/env python
+"""Benchmark of the activation-sparse ReLU FFN forward pass (TwELL) on B200.
+
+One step = one whole layer forward through the C ABI (twell_up_pack: fused
+up-projection + ReLU + TwELL packing; twell_spmm: sparse down-projection) on
+the 1.5B-scale layer (M=4096 tokens, d_model=2048, d_ff=8192, bf16, weights
+N(0, 1/fan_in), bias set for the target activation density, tile_w=128, ell_w
+from the 99th-percentile rule).  Synthetic, seeded inputs; no dataset.
+
+Prints ONE JSON line (rank 0).  Multi-GPU (torchrun): tokens are independent, so
+every rank runs its own 4096-token batch with replicated weights and no
+data-path collective ("scaling": "weak"); value = all ranks' tokens / the
+slowest rank's device time.
+
+--impl reference times the CPU oracle (fp64 NumPy) on the host cores on a
+bounded sample of the same workload; nothing else exists to compare against.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse FFN tokens/s per layer vs activation density; % of roofline (HBM/TC)"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return dict(hbm_gbs=float(j["hbm_gbs"]), tc_tflops=float(j["bf16_tflops"]),
+                    tc_tflops_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, tc_tflops=1590.0, tc_tflops_sustained=1400.0, source="fallback")
+
+
+def _kernel_source_hash(path):
+    with open(os.path.join(ROOT, path), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def _ncu_traffic(kernel_file, workload):
+    """DRAM bytes per launch from the committed ncu summary, only if it was taken
+    on the current source of the kernel (else null)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        j = json.load(fh)
+    e = j.get(workload, {}).get(kernel_file)
+    if not e or e.get("source_sha256_16") != _kernel_source_hash(
+            os.path.join("activation_sparse_ffn_twell_b200", "csrc", kernel_file)):
+        return None
+    return float(e["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            self.h = N.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        N = self.N
+        names = {
+            "gpu_idle": getattr(N, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(N, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(N, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(N, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(N, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(N, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                try:
+                    r = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = N.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(s)}
+
+
+# ---------------------------------------------------------------------------
+def _workload(density, M, seed):
+    import twell_synth as S
+    return S.relu_15b(density=density, M=M, seed=seed)
+
+
+def _roofline_layer(L, nnz_total, touched_rows, peaks):
+    """North-star roofline of the whole layer: max(useful FLOP / TC peak,
+    unavoidable bytes / HBM BW).  Useful FLOP = dense up (x2 if gated) + 2*nnz*d;
+    unavoidable bytes = x + W_up (+W_gate) + b + touched W_down rows + y."""
+    M, d, f = L.M, L.d_model, L.d_ff
+    flop = 2.0 * M * d * f * (2 if L.gated else 1) + 2.0 * nnz_total * d
+    byts = 2.0 * (M * d + f * d * (2 if L.gated else 1) + f + touched_rows * d + M * d)
+    t_tc = flop / (peaks["tc_tflops"] * 1e12)
+    t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+    return dict(t_s=max(t_tc, t_hbm), bound="tensor" if t_tc >= t_hbm else "hbm",
+                useful_flop=flop, unavoidable_bytes=byts)
+
+
+def run_ours(args):
+    import torch
+    import activation_sparse_ffn_twell_b200 as T
+    from activation_sparse_ffn_twell_b200 import dist as D
+
+    rank, local, world = D.init("nccl" if args.gpus > 1 else "gloo")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks = _peaks()
+
+    def to_dev(bits):
+        import numpy as np
+        return None if bits is None else torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    L = _workload(args.density, args.M, seed=args.seed + rank)   # own token batch per rank
+    x, wu, b, wd = to_dev(L.x), to_dev(L.w_up), to_dev(L.b), to_dev(L.w_down)
+    M, d, f, tw, E = L.M, L.d_model, L.d_ff, L.tile_w, L.ell_w
+    T_tiles = f // tw
+    cap = min(M * T_tiles, max(4096, (M * T_tiles) // 8))
+    a = T.TwELL.allocate(M, f, tw, E, cap, device=dev)
+    y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        T.twell_up_pack(x, wu, b, tile_w=tw, ell_w=E, out=a)
+        T.twell_spmm(a, wd, mode=args.mode, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    code, n_ovf = T.read_status(a)
+    if code != 0:
+        raise SystemExit(f"status {T.STATUS[code]} after warm-up")
+    nnz = a.nnz_u16()
+    nnz_total = int(nnz.sum().item())
+    # W_down rows any token touches (hidden units active for at least one token)
+    # are counted from the packed output with a tiny torch reduction off the timed path.
+    touched = int(_touched_rows(a, torch).item())
+    density = nnz_total / float(M * f)
+
+    # ------------------------------------------------ timed region (device events)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    D.barrier(dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()                      # evict L2 between steps (inputs < 126 MB)
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            T.twell_up_pack(x, wu, b, tile_w=tw, ell_w=E, out=a)
+            e1.record(stream)
+            T.twell_spmm(a, wd, mode=args.mode, y=y)
+            e2.record(stream)
+        torch.cuda.synchronize(dev)
+        wall = time.perf_counter() - wall0
+    D.barrier(dev)
+    up_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    down_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    step_ms = sum(u + v for u, v in zip(up_ms, down_ms)) / args.steps
+    step_ms_max = D.max_over_ranks(step_ms, dev if world > 1 and args.gpus > 1 else None)
+    code, n_ovf2 = T.read_status(a)
+    if code != 0:
+        raise SystemExit(f"status {T.STATUS[code]} in timed region")
+
+    tokens_s = world * M / (step_ms_max * 1e-3)
+    up_avg_s = sum(up_ms) / len(up_ms) * 1e-3
+    up_flop = 2.0 * M * d * f
+    achieved_tflops = up_flop / up_avg_s / 1e12
+    rl = _roofline_layer(L, nnz_total, touched, peaks)
+
+    result = {
+        "metric": METRIC, "value": tokens_s, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1/fan_in) weights, bias for target density)",
+        "config": {"workload": "relu_ffn_layer_1.5b", "M": M, "d_model": d, "d_ff": f,
+                   "target_density": args.density, "measured_density": density,
+                   "tile_w": tw, "ell_w": E, "gated": False, "down_mode": args.mode,
+                   "n_ovf": n_ovf, "l2": "flushed: 256 MiB write between timed steps",
+                   "parallelism": f"token-sharded x{world} (weights replicated, no collective)"},
+        "roofline": {"bound": "tensor", "kernel": "k_up_pack (fused up-GEMM + ReLU + TwELL pack)",
+                     "achieved": achieved_tflops, "peak": peaks["tc_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tflops / peaks["tc_tflops"],
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "traffic": _ncu_traffic("k_up_pack.cu", f"relu_15b_rho{args.density:g}"),
+                     "interval": "twell_up_pack call (up kernel + 2 small finalize kernels)",
+                     "up_ms": up_avg_s * 1e3, "down_ms": sum(down_ms) / len(down_ms)},
+        "roofline_layer": {"bound": rl["bound"], "roofline_ms": rl["t_s"] * 1e3,
+                           "frac": rl["t_s"] * 1e3 / step_ms_max,
+                           "useful_flop": rl["useful_flop"],
+                           "unavoidable_bytes": rl["unavoidable_bytes"],
+                           "touched_w_down_rows": touched, "peaks": peaks["source"]},
+        "gpu_launches": args.steps * _kernels_per_step(args.mode),
+        "wall_s_timed_region": wall,
+    }
+    result["clocks"] = clk.summary()
+
+    if not args.quick:
+        result["dense_ffn"] = _dense_baseline(x, wu, b, wd, args, flush, stream, dev)
+        result["e2e"] = _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world)
+        if args.sweep:
+            result["density_sweep"] = _sweep(T, args, dev, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = _cpu_baseline(L, seconds=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    del a
+    D.finish()
+
+
+def _touched_rows(a, torch):
+    # a hidden unit j is touched if any token has it among its packed nonzeros
+    # (ELL slots of non-overflowing pairs, or nonzeros of a backup segment)
+    M, T_, E = a.vals.shape
+    tw = a.tile_w
+    nnz = a.nnz_u16()
+    live = torch.arange(E, device=a.vals.device)[None, None, :] < torch.minimum(nnz, torch.tensor(E, device=nnz.device))[:, :, None]
+    live = live & (nnz[:, :, None] <= E)
+    cols = (torch.arange(T_, device=a.vals.device)[None, :, None] * tw + a.idx.to(torch.int64))
+    touched = torch.zeros(a.d_ff, dtype=torch.bool, device=a.vals.device)
+    touched[cols[live]] = True
+    n = int(a.n_ovf.item())
+    if n:
+        pos = a.ovf_pos[:n].to(torch.int64)
+        t = pos % T_
+        seg = a.ovf_dense[:n].view(torch.int16) & 0x7FFF
+        jj = torch.nonzero(seg != 0)
+        touched[t[jj[:, 0]] * tw + jj[:, 1]] = True
+    return touched.sum()
+
+
+def _kernels_per_step(mode):
+    # up_pack: k_up_pack + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds k_block_path
+    # and launches both down kernels (each skips the token blocks the other owns)
+    return 3 + (3 if mode == "auto" else 1)
+
+
+def _dense_baseline(x, wu, b, wd, args, flush, stream, dev):
+    """Same-shape dense bf16 FFN through cuBLAS (torch.matmul), same run, same timing."""
+    import torch
+    import torch.nn.functional as F
+
+    def dense():
+        h = torch.relu(F.linear(x, wu, b))
+        return torch.matmul(h, wd)
+    for _ in range(max(3, args.warmup)):
+        dense()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dense()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in ts) / len(ts)
+    return {"ms_per_step": ms, "tokens_s": x.shape[0] / (ms * 1e-3),
+            "impl": "torch.matmul bf16 (cuBLAS): relu(x W_up^T + b) W_down"}
+
+
+def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
+    """End to end through the public API with host buffers: pinned x -> device,
+    the layer, y -> pinned host, every step inside the timed region."""
+    import numpy as np
+    import torch
+    from activation_sparse_ffn_twell_b200 import dist as D
+    xh = torch.from_numpy(L.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    yh = torch.empty((L.M, L.d_model), dtype=torch.bfloat16).pin_memory()
+    xd = torch.empty_like(x)
+    for _ in range(3):
+        xd.copy_(xh, non_blocking=True)
+        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=args.mode, out=a, y=y)
+        yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=args.mode, out=a, y=y)
+        yh.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = D.max_over_ranks(ms, dev if world > 1 else None)
+    return {"value": world * L.M / (ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": int(L.M * L.d_model * 2),
+            "d2h_bytes_per_step": int(L.M * L.d_model * 2),
+            "ms_per_step": ms, "note": "weights resident; x in / y out through pinned host memory"}
+
+
+def _sweep(T, args, dev, peaks):
+    import numpy as np
+    import torch
+    import torch.nn.functional as F
+    out = []
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for rho in (0.20, 0.10, 0.05, 0.01):
+        L = _workload(rho, args.M, args.seed)
+        tb = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        x, wu, b, wd = tb(L.x), tb(L.w_up), tb(L.b), tb(L.w_down)
+        T_tiles = L.d_ff // L.tile_w
+        a = T.TwELL.allocate(L.M, L.d_ff, L.tile_w, L.ell_w,
+                             min(L.M * T_tiles, max(4096, L.M * T_tiles // 8)), device=dev)
+        y = torch.empty((L.M, L.d_model), dtype=torch.bfloat16, device=dev)
+        row = {"target_density": rho, "ell_w": L.ell_w}
+        for mode in ("auto", "gather", "mma"):
+            for _ in range(3):
+                T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=mode, out=a, y=y)
+            evs = []
+            for _ in range(max(5, args.steps // 4)):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=mode, out=a, y=y)
+                e1.record()
+                evs.append((e0, e1))
+            torch.cuda.synchronize(dev)
+            row[f"{mode}_ms"] = sum(p.elapsed_time(q) for p, q in evs) / len(evs)
+        code, n_ovf = T.read_status(a)
+        nnz_total = int(a.nnz_u16().sum().item())
+        row["measured_density"] = nnz_total / float(L.M * L.d_ff)
+        row["n_ovf"] = n_ovf
+        rl = _roofline_layer(L, nnz_total, int(_touched_rows(a, torch).item()), peaks)
+        best = min(row["auto_ms"], row["gather_ms"], row["mma_ms"])
+        row["roofline_ms"] = rl["t_s"] * 1e3
+        row["frac_roofline_auto"] = rl["t_s"] * 1e3 / row["auto_ms"]
+        row["tokens_s_auto"] = L.M / (row["auto_ms"] * 1e-3)
+        # dense comparator
+        for _ in range(3):
+            torch.matmul(torch.relu(F.linear(x, wu, b)), wd)
+        evs = []
+        for _ in range(max(5, args.steps // 4)):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(torch.relu(F.linear(x, wu, b)), wd)
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        row["dense_ms"] = sum(p.elapsed_time(q) for p, q in evs) / len(evs)
+        row["speedup_vs_dense_auto"] = row["dense_ms"] / row["auto_ms"]
+        row["best_ms"] = best
+        out.append(row)
+        del a, x, wu, b, wd, y
+    return out
+
+
+# ---------------------------------------------------------------------------
+def _cpu_baseline(L, seconds=10.0, sample_tokens=256):
+    """The oracle, as it stands, on the host cores over a bounded token sample of
+    the same layer (full weights); repeats the sample until ~`seconds` elapse."""
+    import numpy as np
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    done, t0 = 0, time.perf_counter()
+    reps = 0
+    while True:
+        r0 = (reps * sample_tokens) % L.M
+        rows = slice(r0, r0 + sample_tokens)
+        O.ffn_forward(L.x[rows], L.w_up, L.b, L.w_down, L.tile_w, L.ell_w)
+        done += min(sample_tokens, L.M - r0)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 64:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{reps} x {sample_tokens}-token slices of the {L.M}-token batch, full "
+                      f"{L.d_model}x{L.d_ff} weights, fp64 NumPy, {el:.1f} s"}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    from activation_sparse_ffn_twell_b200 import dist as D
+    rank, _, world = D.env_rank_world()
+    if rank != 0:
+        return
+    L = _workload(args.density, args.M, args.seed)
+    for _ in range(args.warmup):
+        _cpu_baseline(L, seconds=0.0, sample_tokens=64)
+    per = []
+    for _ in range(args.steps):
+        cb = _cpu_baseline(L, seconds=0.0, sample_tokens=args.ref_tokens)
+        per.append(cb)
+    value = sum(c["value"] for c in per) / len(per)
+    ms = args.ref_tokens / value * 1e3 * (L.M / args.ref_tokens)
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "impl": "reference", "device": "cpu (host cores)",
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "relu_ffn_layer_1.5b", "M": L.M, "d_model": L.d_model,
+                   "d_ff": L.d_ff, "target_density": args.density, "tile_w": L.tile_w,
+                   "ell_w": L.ell_w},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per[0]["cores"], "kind": "oracle",
+                         "sample": f"each step: {args.ref_tokens} tokens of the {L.M}-token batch"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--density", type=float, default=0.05)
+    ap.add_argument("--M", type=int, default=4096)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--mode", default="auto", choices=["auto", "gather", "mma"])
+    ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")
+    ap.add_argument("--quick", action="store_true", help="skip dense/e2e legs (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-tokens", type=int, default=128)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,157 @@
+/*
+ * twell.h -- C ABI of the B200 (sm_100a) activation-sparse FFN library.
+ *
+ * The operation is the forward pass of a ReLU feed-forward layer whose hidden
+ * activations are mostly zero: an up-projection to a wide hidden dimension, a
+ * ReLU, and a down-projection back to the model dimension, tokens independent
+ * ("Sparser, Faster, Lighter Transformer Language Models", Sakana AI / NVIDIA;
+ * upppp.jp 2026-05-11, section 「LLMフィードフォワード層の「無駄」とは何か」).
+ * The hidden activations are packed into TwELL (Tile-wise ELLPACK): hidden
+ * columns are cut into fixed-width tiles and, per token and tile, an ELL list of
+ * (value, in-tile index) slots keeps the nonzeros; (token, tile) pairs with more
+ * nonzeros than the ELL width also keep their dense tile segment in a small dense
+ * backup -- the "hybrid" sparse-main plus dense-backup form (same page, section
+ * 「TwELLとカスタムCUDAカーネルが解決する課題」).  The down-projection reads only
+ * the packed form.
+ *
+ * Conventions for every call
+ *  - bf16 tensors are passed as uint16_t bit patterns.  All tensor pointers are
+ *    DEVICE pointers, caller-owned, 16-byte aligned, row-major and dense unless a
+ *    leading dimension says otherwise.  The library allocates no device memory;
+ *    scratch comes from the caller's workspace (see twell_workspace_bytes).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous: they validate arguments on the host, enqueue kernels and
+ *    return.  Argument errors are returned before anything is enqueued.
+ *  - Asynchronous errors (backup capacity exhausted, a bounded device wait that
+ *    timed out) are recorded in the matrix's device status word; read them with
+ *    twell_read_status, which synchronises the stream.
+ *  - Shapes: tile_w in {32, 64, 128, 256}; d_ff % tile_w == 0;
+ *    1 <= ell_w <= tile_w; d_model % 64 == 0; M >= 0 (M == 0 is a no-op).
+ */
+#ifndef TWELL_B200_H
+#define TWELL_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TWELL_OK = 0,
+  TWELL_ERR_INVALID_ARG = 1,      /* null/misaligned pointer, bad shape            */
+  TWELL_ERR_UNSUPPORTED = 2,      /* legal but not implemented (e.g. gated tile_w 256) */
+  TWELL_ERR_OVERFLOW_CAPACITY = 3,/* async: more overflow pairs than ovf_capacity   */
+  TWELL_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed               */
+  TWELL_ERR_TIMEOUT = 5,          /* async: a bounded device wait gave up            */
+  TWELL_ERR_WORKSPACE = 6         /* workspace missing or smaller than required      */
+} twell_status;
+
+/* Down-projection path selection. */
+typedef enum {
+  TWELL_DOWN_AUTO = 0,   /* per 128-token block, by measured density crossover   */
+  TWELL_DOWN_GATHER = 1, /* CUDA-core gather of W_down rows per packed nonzero    */
+  TWELL_DOWN_MMA = 2     /* tcgen05 tensor cores on h tiles rebuilt from TwELL    */
+} twell_down_mode;
+
+/*
+ * A TwELL matrix of M tokens x d_ff hidden units (T = d_ff / tile_w tiles).
+ *   vals      [M][T][ell_w]  bf16  slot values; unused slots hold +0
+ *   idx       [M][T][ell_w]  u8    in-tile column of each slot (unused: 0)
+ *   nnz       [M][T]         u16   TRUE nonzero count of the pair (may exceed ell_w)
+ *   n_ovf     [1]            i32   number of pairs with nnz > ell_w (true count)
+ *   ovf_pos   [ovf_capacity] i32   r*T + t of each overflowing pair, ascending
+ *   ovf_dense [ovf_capacity][tile_w] bf16  the pair's whole dense tile segment
+ *   status    [1]            i32   0, or a twell_status raised on the device
+ * Slots list a pair's nonzeros in ascending in-tile order; "nonzero" means the
+ * bf16 value is not +-0, and every stored zero is +0.  For an overflowing pair the
+ * slots still hold its first ell_w nonzeros; consumers use the dense segment.
+ * All arrays are device memory owned by the caller.
+ */
+typedef struct {
+  int32_t M, d_ff, tile_w, ell_w;
+  uint16_t *vals;
+  uint8_t *idx;
+  uint16_t *nnz;
+  int32_t ovf_capacity;
+  int32_t *n_ovf;
+  int32_t *ovf_pos;
+  uint16_t *ovf_dense;
+  int32_t *status;
+} twell_matrix;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int twell_version(void);
+
+/* Human-readable name of a status code (static string). */
+const char *twell_status_string(twell_status s);
+
+/*
+ * Workspace bytes needed by twell_pack / twell_up_pack / twell_spmm /
+ * twell_ffn_forward for these sizes (the maximum over the four calls).  gated is
+ * 0 or 1.  Returns 0 for invalid shapes.
+ */
+size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w, int gated,
+                             int ovf_capacity);
+
+/*
+ * twell_pack -- dense hidden activations h -> TwELL (+ dense backup).
+ *   h      [M][ld_h] bf16 (ld_h >= d_ff, ld_h % 8 == 0); only columns < d_ff are read.
+ *   out    fully described destination matrix (out->M, d_ff, tile_w, ell_w must
+ *          equal the arguments).  Every field of *out is written.
+ * The TwELL definition is the one above (upppp.jp 2026-05-11, TwELL section).
+ */
+twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
+                        const twell_matrix *out, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * twell_up_pack -- the fused producer: z = x W_up^T (+ b), h = bf16(ReLU(z)),
+ * or gated h = bf16(ReLU(x W_gate^T + b) * (x W_up^T)), written straight into
+ * TwELL without a dense h in memory ("builds TwELL on the fly", upppp.jp
+ * 2026-05-11, TwELL section).
+ *   x       [M][d_model] bf16
+ *   W_up    [d_ff][d_model] bf16 (row j = hidden unit j)
+ *   W_gate  [d_ff][d_model] bf16 or NULL (non-gated)
+ *   b       [d_ff] bf16 or NULL; with W_gate it is the gate bias
+ *   z_debug NULL, or fp32 [M][d_ff] (non-gated: x W_up^T before the bias) /
+ *           [M][2*d_ff] (gated: per row, d_ff gate values then d_ff up values).
+ *           Test hook: lets a caller re-derive h exactly from the GPU's own fp32
+ *           accumulators.
+ * Gated requires tile_w <= 128.  ell_w <= 64 on this fused path.
+ */
+twell_status twell_up_pack(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                           const uint16_t *b, int M, int d_model, int d_ff, int tile_w,
+                           int ell_w, const twell_matrix *out, float *z_debug, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/*
+ * twell_spmm -- y = h W_down reading h only from TwELL + backup.
+ *   W_down [d_ff][d_model] bf16 (row j = hidden unit j's output vector)
+ *   y      [M][d_model] bf16 (fp32 accumulation, one rounding at the end)
+ *   mode   a twell_down_mode.
+ * If the matrix's status word holds TWELL_ERR_OVERFLOW_CAPACITY, y is undefined.
+ */
+twell_status twell_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model,
+                        uint16_t *y, int mode, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * twell_ffn_forward -- the whole layer: twell_up_pack followed by twell_spmm on
+ * the same stream.  `twell` receives the packed activations (it is the
+ * intermediate, left populated).  Arguments as in the two calls above.
+ */
+twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                               const uint16_t *b, const uint16_t *W_down, int M, int d_model,
+                               int d_ff, int tile_w, int ell_w, const twell_matrix *twell,
+                               uint16_t *y, int mode, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronise `stream`, then return the matrix's device status word (TWELL_OK if
+ * clean) and, if n_ovf_out is not NULL, the true overflow-pair count.
+ */
+twell_status twell_read_status(const twell_matrix *a, void *stream, int32_t *n_ovf_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TWELL_B200_H */

@@ -270,7 +270,9 @@ def small_random(M: int, d_model: int, d_ff: int, tile_w: int, ell_w: int, densi
     elif density <= 0.0:
         b = bf16_bits_from_f32(np.full(d_ff, -1.0e4, dtype=np.float32))
     elif density >= 1.0:
-        b = bf16_bits_from_f32(np.full(d_ff, 1.0e4, dtype=np.float32))
+        # +6 sigma: every pre-activation is positive (P < 1e-9 otherwise) while h,
+        # and therefore y, stay O(1)
+        b = bf16_bits_from_f32((6.0 * _row_norms(src)).astype(np.float32))
     else:
         b = _bias_for_density(_row_norms(src), density)
     return FFNInputs(f"small_M{M}_d{d_model}_f{d_ff}_tw{tile_w}_E{ell_w}", M, d_model, d_ff,
