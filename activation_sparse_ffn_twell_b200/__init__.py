@@ -24,7 +24,7 @@ from typing import Optional
 __all__ = [
     "TwellError", "TwELL", "lib", "library_path", "workspace_bytes",
     "twell_pack", "twell_up_pack", "twell_spmm", "twell_ffn_forward", "read_status",
-    "DOWN_MODES", "STATUS",
+    "DOWN_MODES", "STATUS", "default_ovf_capacity",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -122,6 +122,12 @@ def _need_bf16(name, t, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def default_ovf_capacity(M: int, n_tiles: int) -> int:
+    """Backup capacity used when the caller gives none: 1/8 of all (token, tile)
+    pairs, at least 4096 pairs, never more than all of them."""
+    return min(M * n_tiles, max(4096, (M * n_tiles) // 8))
+
+
 @dataclasses.dataclass
 class TwELL:
     """A TwELL matrix in device memory (torch tensors) plus its dense backup."""
@@ -149,7 +155,7 @@ class TwELL:
         torch = _torch()
         T = d_ff // tile_w
         if ovf_capacity is None:
-            ovf_capacity = min(M * T, max(1024, (M * T + 7) // 8))
+            ovf_capacity = default_ovf_capacity(M, T)
         dev = device if device is not None else torch.device("cuda")
         cap_alloc = max(ovf_capacity, 1)
         return TwELL(M, d_ff, tile_w, ell_w, ovf_capacity,

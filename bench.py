@@ -167,8 +167,7 @@ def run_ours(args):
     x, wu, b, wd = to_dev(L.x), to_dev(L.w_up), to_dev(L.b), to_dev(L.w_down)
     M, d, f, tw, E = L.M, L.d_model, L.d_ff, L.tile_w, L.ell_w
     T_tiles = f // tw
-    cap = min(M * T_tiles, max(4096, (M * T_tiles) // 8))
-    a = T.TwELL.allocate(M, f, tw, E, cap, device=dev)
+    a = T.TwELL.allocate(M, f, tw, E, T.default_ovf_capacity(M, T_tiles), device=dev)
     y = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -354,8 +353,8 @@ def _sweep(T, args, dev, peaks):
         tb = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
         x, wu, b, wd = tb(L.x), tb(L.w_up), tb(L.b), tb(L.w_down)
         T_tiles = L.d_ff // L.tile_w
-        a = T.TwELL.allocate(L.M, L.d_ff, L.tile_w, L.ell_w,
-                             min(L.M * T_tiles, max(4096, L.M * T_tiles // 8)), device=dev)
+        a = T.TwELL.allocate(L.M, L.d_ff, L.tile_w, L.ell_w, T.default_ovf_capacity(L.M, T_tiles),
+                             device=dev)
         y = torch.empty((L.M, L.d_model), dtype=torch.bfloat16, device=dev)
         row = {"target_density": rho, "ell_w": L.ell_w}
         for mode in ("auto", "gather", "mma"):

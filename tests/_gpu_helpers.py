@@ -67,11 +67,18 @@ def assert_twell_valid(a):
 
 
 def y_errors(y_gpu, y_ref):
+    """(relative L2 error, max abs error beyond the output-rounding allowance).
+
+    The absolute bound 3e-2 is met by any correct bf16 result only while |y| < 8
+    (half a bf16 ulp is 2^-9 |y|); where |y_ref| is larger, one bf16 ulp of y_ref
+    is allowed instead, so the bound never asks for more than bf16 can store."""
     yg = y_gpu.float().cpu().numpy().astype(np.float64)
-    diff = yg - y_ref
+    diff = np.abs(yg - y_ref)
     nrm = np.linalg.norm(y_ref)
     rel = np.linalg.norm(diff) / nrm if nrm > 0 else (0.0 if np.all(yg == 0) else np.inf)
-    return rel, float(np.max(np.abs(diff))) if diff.size else 0.0
+    allow = np.maximum(Y_MAX_ABS, 2.0 ** -8 * np.abs(y_ref))
+    excess = float(np.max(diff - allow + Y_MAX_ABS)) if diff.size else 0.0
+    return rel, excess
 
 
 def assert_y_close(y_gpu, y_ref):
