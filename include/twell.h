@@ -146,6 +146,32 @@ twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const ui
                                uint16_t *y, int mode, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * twell_pack_noalloc -- twell_pack for callers that cannot provide a workspace.
+ * The paper has no counterpart to this call; it exists for deployment.
+ *
+ * twell_pack needs caller-owned scratch.  Callers that cannot allocate device
+ * memory when they pack -- a serving runtime that reserved the whole GPU up front
+ * and forbids cudaMalloc on its request path, or a plugin interface that hands
+ * over only input and output buffers -- use this variant instead.  It takes the
+ * same arguments minus the workspace, produces the same output, and allocates
+ * nothing: its scratch is a fixed 4 MiB device array inside the library, which
+ * every GPU that loads the library holds until the process exits.
+ *   - Scratch needed: 64 + 8*M + ovf_capacity*(4 + 2*tile_w) bytes, each part
+ *     rounded up to 256.  A call needing more than 4 MiB returns
+ *     TWELL_ERR_WORKSPACE without doing anything (e.g. M = 4096, tile_w = 128
+ *     allows ovf_capacity up to about 15,900).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current).  Make that first call before any CUDA
+ *     stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents;
+ *     each call clears what must start at zero.  Calls whose executions overlap
+ *     on the GPU (different streams, or different host threads, without ordering
+ *     between them) race on the array and give undefined results.
+ */
+twell_status twell_pack_noalloc(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w,
+                                int ell_w, const twell_matrix *out, void *stream);
+
+/*
  * Synchronise `stream`, then return the matrix's device status word (TWELL_OK if
  * clean) and, if n_ovf_out is not NULL, the true overflow-pair count.
  */
