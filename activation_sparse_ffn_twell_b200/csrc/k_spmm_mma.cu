@@ -13,15 +13,20 @@
 //               swizzle; this is an N-major ("MN-major") B operand.
 //   warp 1      TMEM allocation (2 x 256 fp32 columns) + tcgen05.mma issue.
 //   warps 2..5  epilogue: TMEM -> fp32 registers -> bf16 -> y.
-//   warps 6..9  A builders: thread = token row; zero the row's 128 bytes, then
-//               scatter its slot values (or copy its backup segment) into the
-//               K-major 128-byte-swizzled tile, fence to the async proxy, arrive.
+//   warps 6..9  A builders: thread = token row.  Fast path (ell_w % 8 == 0):
+//               the row's slot record of the next hidden tile is loaded into
+//               registers with 128/64-bit loads while the current one is used;
+//               the K steps of one tile are claimed together, zeroed with
+//               bank-conflict-free 16-byte stores, and each slot is written once
+//               with a predicated 2-byte store (fully unrolled over ell_w).
+//               General path: per K step, zero the row and scatter from global
+//               memory.  Then fence to the async proxy and arrive.
 #include "twell_device.cuh"
 
 namespace twell {
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kMaxStages = 4;
 constexpr int kBN = 256;                        // y columns per tile
 constexpr int kABytes = kBlockM * kBlockK * 2;  // 16 KB
 constexpr int kBBytes = kBlockK * kBN * 2;      // 32 KB (4 boxes of 64 x 64)
@@ -33,6 +38,7 @@ struct DownParams {
   uint16_t *y;
   int d;
   int num_m_blocks, num_n_blocks, num_kb;
+  int stages;                // pipeline depth (<= kMaxStages), set from shared-memory budget
   const int32_t *blk_path;   // NULL, or per 128-token block: 1 = this path owns it
 };
 
@@ -51,20 +57,22 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
   return P.blk_path == nullptr || P.blk_path[m_blk] != 0;
 }
 
+template <int EV>   // ell_w / 8 on the fast builder path, 0 = general path
 __global__ void __launch_bounds__(kThreads, 1)
     k_spmm_mma(const __grid_constant__ CUtensorMap tmap_wd, const DownParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int kStages = P.stages;
   uint8_t *sA = smem;
   uint8_t *sB = smem + kStages * kABytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBBytes);
   uint64_t *full = bars;
-  uint64_t *empty = bars + kStages;
-  uint64_t *tm_full = bars + 2 * kStages;
-  uint64_t *tm_empty = bars + 2 * kStages + 2;
-  uint64_t *drain = bars + 2 * kStages + 4;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kStages + 5);
+  uint64_t *empty = bars + kMaxStages;
+  uint64_t *tm_full = bars + 2 * kMaxStages;
+  uint64_t *tm_empty = bars + 2 * kMaxStages + 2;
+  uint64_t *drain = bars + 2 * kMaxStages + 4;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kMaxStages + 5);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -200,8 +208,128 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&tm_empty[acc]);
     }
+  } else if constexpr (EV > 0) {
+    // ------------------------------------------------------------ A builders (fast)
+    // ell_w == 8*EV.  Per hidden tile, the row's slot record (values, indices,
+    // nnz) is loaded into registers one tile ahead; the tile's K steps are zeroed
+    // with independent 16-byte stores and every slot is written once with a
+    // predicated 2-byte store -- a fully unrolled, dependency-free sequence.
+    constexpr int E = 8 * EV;
+    const int row_in_tile = (warp - 6) * 32 + lane;
+    const int tw = A.tw, Tn = A.T;
+    const int lg_tw = 31 - __clz(tw);
+    const int n_ovf = min(*A.n_ovf, A.cap);
+    const uint32_t row_swz = static_cast<uint32_t>(row_in_tile & 7);
+    int stage = 0; uint32_t phase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int m_blk = tile % P.num_m_blocks;
+      if (!tile_owned(P, m_blk)) continue;
+      const int r = m_blk * kBlockM + row_in_tile;
+      const bool valid = r < A.M;
+      const size_t pair0 = static_cast<size_t>(valid ? r : 0) * Tn;
+
+      // tile t's slot record of this row, straight into registers
+      auto fetch = [&](int t, uint4 (&v)[EV], uint2 (&ix)[EV], int &n) {
+        if (valid && t < Tn) {
+          const uint4 *gv = reinterpret_cast<const uint4 *>(A.vals + (pair0 + t) * E);
+          const uint2 *gi = reinterpret_cast<const uint2 *>(A.idx + (pair0 + t) * E);
+#pragma unroll
+          for (int g = 0; g < EV; ++g) { v[g] = __ldg(gv + g); ix[g] = __ldg(gi + g); }
+          n = static_cast<int>(__ldg(A.nnz + pair0 + t));
+        } else {
+          n = 0;
+        }
+      };
+
+      int cur_t = -1, n0 = 0, n1 = 0, ovf_k = -1;
+      uint4 vq[EV], vq1[EV];
+      uint2 iq[EV], iq1[EV];
+      // K-steps are claimed in groups of S (all steps of one hidden tile when
+      // the ring holds them) so every slot is visited once per tile
+      // (at most stages-1 of them, so the MMA always has a stage to work on)
+      const int S = max(1, min(tw / kBlockK, kStages - 1));
+      for (int kb0 = 0; kb0 < P.num_kb && ok; kb0 += S) {
+        const int nsteps = min(S, P.num_kb - kb0);
+        const int stage0 = stage;
+        for (int j = 0; j < nsteps; ++j) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t *rowA = sA + stage * kABytes + row_in_tile * 128;
+          // Rows are 128 B apart, so lanes storing the same chunk index would all
+          // hit the same 4 banks; row-XOR chunk order makes the zeroing conflict-free.
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            reinterpret_cast<uint4 *>(rowA)[c ^ static_cast<int>(row_swz)] = make_uint4(0, 0, 0, 0);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        const int col0 = kb0 * kBlockK, span = nsteps * kBlockK;
+        const int t_last = (col0 + span - 1) >> lg_tw;
+        for (int t = col0 >> lg_tw; t <= t_last; ++t) {   // 1 tile, or 2 when tile_w == 32
+          if (t != cur_t) {                                // same for every thread of the CTA
+            if (cur_t < 0) {
+              fetch(t, vq, iq, n0);
+            } else {
+#pragma unroll
+              for (int g = 0; g < EV; ++g) { vq[g] = vq1[g]; iq[g] = iq1[g]; }
+              n0 = n1;
+            }
+            fetch(t + 1, vq1, iq1, n1);                    // one tile ahead; used next advance
+            cur_t = t;
+            ovf_k = (n0 > E) ? find_ovf(A.ovf_pos, n_ovf, static_cast<int>(pair0) + t) : -1;
+          }
+          if (!valid || t >= Tn || n0 == 0) continue;
+          const int base = (t << lg_tw) - col0;           // group column of in-tile index 0
+          if (n0 <= E) {
+#pragma unroll
+            for (int g = 0; g < EV; ++g) {
+              const uint32_t vw[4] = {vq[g].x, vq[g].y, vq[g].z, vq[g].w};
+              const uint32_t iw[2] = {iq[g].x, iq[g].y};
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int sl = 8 * g + k;
+                const uint32_t col = static_cast<uint32_t>(base + static_cast<int>((iw[k >> 2] >> (8 * (k & 3))) & 0xFFu));
+                if (sl < n0 && col < static_cast<uint32_t>(span)) {
+                  int sb = stage0 + static_cast<int>(col >> 6);   // step buffer of this column
+                  if (sb >= kStages) sb -= kStages;
+                  const uint32_t c = col & 63u;
+                  const uint32_t off = (((c >> 3) ^ row_swz) << 4) + ((c & 7u) << 1);
+                  *reinterpret_cast<uint16_t *>(sA + sb * kABytes + row_in_tile * 128 + off) =
+                      static_cast<uint16_t>((k & 1) ? (vw[k >> 1] >> 16) : (vw[k >> 1] & 0xFFFFu));
+                }
+              }
+            }
+          } else if (ovf_k >= 0) {                        // dense backup segment
+            // group columns c with in-tile index c - base inside [0, tile_w)
+            const int lo = max(0, base), hi = min(span, base + tw);
+            for (int c = lo; c < hi; c += 8) {
+              const uint4 q = __ldg(reinterpret_cast<const uint4 *>(
+                  A.ovf_dense + static_cast<size_t>(ovf_k) * tw + (c - base)));
+              int sb = stage0 + (c >> 6);
+              if (sb >= kStages) sb -= kStages;
+              const uint32_t cc = static_cast<uint32_t>(c & 63);
+              *reinterpret_cast<uint4 *>(sA + sb * kABytes + row_in_tile * 128 +
+                                         (((cc >> 3) ^ row_swz) << 4)) = q;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int j = 0; j < nsteps; ++j) {
+            int sb = stage0 + j;
+            if (sb >= kStages) sb -= kStages;
+            mbar_arrive(&full[sb]);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      raise_status(A.status, TWELL_ERR_TIMEOUT);
+    }
   } else {
-    // ------------------------------------------------------------ A builders
+    // ------------------------------------------------------------ A builders (general)
     const int row_in_tile = (warp - 6) * 32 + lane;
     const int n_ovf = min(*A.n_ovf, A.cap);
     int stage = 0; uint32_t phase = 0;
@@ -216,7 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *tileA = sA + stage * kABytes;
         uint8_t *rowA = tileA + row_in_tile * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(rowA)[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < 8; ++c)   // row-XOR chunk order: conflict-free across the warp
+          reinterpret_cast<uint4 *>(rowA)[c ^ (row_in_tile & 7)] = make_uint4(0, 0, 0, 0);
         if (valid) {
           const int k0 = kb * kBlockK;               // first hidden column of this stage
           for (int t = k0 / A.tw; t * A.tw < k0 + kBlockK && t < A.T; ++t) {
@@ -291,6 +420,16 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
   }
 }
 
+template <int EV>
+cudaError_t launch_down(const CUtensorMap &mw, const DownParams &P, int grid, size_t smem,
+                        cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(k_spmm_mma<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  k_spmm_mma<EV><<<grid, kThreads, smem, s>>>(mw, P);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s) {
@@ -315,14 +454,27 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   P.num_n_blocks = (d + kBN - 1) / kBN;
   P.num_kb = (v.f + kBlockK - 1) / kBlockK;
   P.blk_path = blk_path;
-  const size_t smem = 1024 + kStages * (kABytes + kBBytes) + 256;
-  cudaError_t e = cudaFuncSetAttribute(k_spmm_mma, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  const int ev = (v.E % 8 == 0 && v.E <= 64) ? v.E / 8 : 0;
+  const size_t fixed = 1024 + 256;
+  const size_t budget = 227 * 1024;
+  int stages = static_cast<int>((budget - fixed) / (kABytes + kBBytes));
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages < 2) return cudaErrorInvalidValue;
+  P.stages = stages;
+  const size_t smem = fixed + static_cast<size_t>(stages) * (kABytes + kBBytes);
   const int tiles = P.num_m_blocks * P.num_n_blocks;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k_spmm_mma<<<grid, kThreads, smem, s>>>(mw, P);
-  return cudaGetLastError();
+  switch (ev) {
+    case 1: return launch_down<1>(mw, P, grid, smem, s);
+    case 2: return launch_down<2>(mw, P, grid, smem, s);
+    case 3: return launch_down<3>(mw, P, grid, smem, s);
+    case 4: return launch_down<4>(mw, P, grid, smem, s);
+    case 5: return launch_down<5>(mw, P, grid, smem, s);
+    case 6: return launch_down<6>(mw, P, grid, smem, s);
+    case 7: return launch_down<7>(mw, P, grid, smem, s);
+    case 8: return launch_down<8>(mw, P, grid, smem, s);
+    default: return launch_down<0>(mw, P, grid, smem, s);
+  }
 }
 
 }  // namespace twell
