@@ -16,22 +16,30 @@
 //   warps 6..9  A builders: thread = token row.  Fast path (ell_w % 8 == 0):
 //               the row's slot record of the next hidden tile is loaded into
 //               registers with 128/64-bit loads while the current one is used;
-//               the K steps of one tile are claimed together, zeroed with
-//               bank-conflict-free 16-byte stores, and each slot is written once
-//               with a predicated 2-byte store (fully unrolled over ell_w).
+//               the K steps of one tile are claimed together (the TMA warp
+//               has already cleared them with a bulk copy of zeros), and each
+//               slot is written once with a predicated 2-byte store (fully
+//               unrolled over ell_w).
 //               General path: per K step, zero the row and scatter from global
 //               memory.  Then fence to the async proxy and arrive.
+#include <cstdlib>
+
 #include "twell_device.cuh"
 
 namespace twell {
 namespace {
 
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kBN = 256;                        // y columns per tile
 constexpr int kABytes = kBlockM * kBlockK * 2;  // 16 KB
 constexpr int kBBytes = kBlockK * kBN * 2;      // 32 KB (4 boxes of 64 x 64)
-constexpr int kThreads = 320;
-constexpr uint32_t kIdesc = idesc_bf16_f32(kBlockM, kBN, 0, 1);   // A K-major, B N-major
+constexpr int kThreads = 352;
+constexpr int kSlotRing = 4;                    // slot-record ring depth (hidden tiles)
+
+// Source of the per-stage A clear: the fast builders only write nonzeros, the
+// TMA engine zeroes the stage first (a bulk copy from this never-written array),
+// which keeps 16 KB per K step off the threads' shared-memory store path.
+__device__ __align__(128) uint8_t g_zero_tile[kBlockM * kBlockK * 2];
 
 struct DownParams {
   TwellView A;
@@ -39,6 +47,7 @@ struct DownParams {
   int d;
   int num_m_blocks, num_n_blocks, num_kb;
   int stages;                // pipeline depth (<= kMaxStages), set from shared-memory budget
+  int slot_ib;               // bytes of the index box per row (covers ell_w indices)
   const int32_t *blk_path;   // NULL, or per 128-token block: 1 = this path owns it
 };
 
@@ -57,63 +66,99 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
   return P.blk_path == nullptr || P.blk_path[m_blk] != 0;
 }
 
-template <int EV>   // ell_w / 8 on the fast builder path, 0 = general path
+// EV: ell_w / 8 on the fast builder path, 0 = general path.
+// TSLOT: slot records arrive by TMA into a shared-memory ring (else per-thread loads).
+// PAIR: a cluster of 2 CTAs computes a 256-token x 256-column tile with M=256
+// MMAs (cta_group::2); each CTA builds its 128 rows of A and loads half of the
+// W_down columns, so each SM carries half the B operand traffic.
+template <int EV, bool TSLOT, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-    k_spmm_mma(const __grid_constant__ CUtensorMap tmap_wd, const DownParams P) {
+    k_spmm_mma(const __grid_constant__ CUtensorMap tmap_wd, const __grid_constant__ CUtensorMap tmap_sv,
+               const __grid_constant__ CUtensorMap tmap_si, const __grid_constant__ CUtensorMap tmap_sn,
+               const DownParams P) {
+  constexpr int TILE_M = PAIR ? 2 * kBlockM : kBlockM;
+  constexpr int B_BYTES = PAIR ? kBBytes / 2 : kBBytes;      // this CTA's W_down columns
+  constexpr int B_BOXES = PAIR ? kBN / 128 : kBN / 64;        // 64-column TMA boxes per CTA
+  constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, kBN, 0, 1);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int kStages = P.stages;
   uint8_t *sA = smem;
   uint8_t *sB = smem + kStages * kABytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * kBBytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * B_BYTES);
   uint64_t *full = bars;
   uint64_t *empty = bars + kMaxStages;
   uint64_t *tm_full = bars + 2 * kMaxStages;
   uint64_t *tm_empty = bars + 2 * kMaxStages + 2;
   uint64_t *drain = bars + 2 * kMaxStages + 4;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kMaxStages + 5);
+  uint64_t *s_full = bars + 2 * kMaxStages + 5;               // slot ring
+  uint64_t *s_empty = s_full + kSlotRing;
+  uint64_t *zfull = s_empty + kSlotRing;                        // A stage cleared by TMA
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(zfull + kMaxStages);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  // slot ring entry: [128][ell_w] bf16 values, [128][slot_ib] u8 indices, [128][8] u16 nnz
+  uint8_t *sRing = reinterpret_cast<uint8_t *>(bars) + 512;
+  const int ring_v = kBlockM * 2 * P.A.E, ring_i = kBlockM * P.slot_ib;
+  const int ring_entry = ring_v + ring_i + kBlockM * 16;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const TwellView &A = P.A;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], 1 + 4); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], 4); }
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], 1 + (PAIR ? 8 : 4)); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], PAIR ? 8 : 4); }
+    for (int i = 0; i < kSlotRing; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4); }
+    for (int i = 0; i < kStages; ++i) mbar_init(&zfull[i], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmap_wd);
+    if (TSLOT) { tma_prefetch_desc(&tmap_sv); tma_prefetch_desc(&tmap_si); tma_prefetch_desc(&tmap_sn); }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    if constexpr (PAIR) { tmem_alloc_pair(tmem_slot, 512); tmem_relinquish_pair(); }
+    else { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_tiles = P.num_m_blocks * P.num_n_blocks;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
+  const int row_base = static_cast<int>(rank) * kBlockM;   // this CTA's rows inside a tile
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA (W_down)
     if (lane == 0) {
       int stage = 0; uint32_t phase = 0; uint32_t filled = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
         const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
-        if (!tile_owned(P, m_blk)) continue;
+        if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], kBBytes);
+          if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * B_BYTES);
           filled |= 1u << stage;
-          uint8_t *dst = sB + stage * kBBytes;
+          if constexpr (EV > 0) {   // clear this CTA's A stage for its builders
+            mbar_arrive_expect_tx(&zfull[stage], kABytes);
+            bulk_load(sA + stage * kABytes, g_zero_tile, kABytes, &zfull[stage]);
+          }
+          uint8_t *dst = sB + stage * B_BYTES;
+          const int col_b = n_blk * kBN + static_cast<int>(rank) * (B_BOXES * 64);
 #pragma unroll
-          for (int j = 0; j < kBN / 64; ++j)
-            tma_load_2d(dst + j * (kBlockK * 128), &tmap_wd, &full[stage], n_blk * kBN + j * 64,
-                        kb * kBlockK);
+          for (int j = 0; j < B_BOXES; ++j) {
+            if constexpr (PAIR)
+              tma_load_2d_pair(dst + j * (kBlockK * 128), &tmap_wd, map_to_cta(&full[stage], 0),
+                               col_b + j * 64, kb * kBlockK);
+            else
+              tma_load_2d(dst + j * (kBlockK * 128), &tmap_wd, &full[stage], col_b + j * 64,
+                          kb * kBlockK);
+          }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -122,67 +167,101 @@ __global__ void __launch_bounds__(kThreads, 1)
         raise_status(A.status, TWELL_ERR_TIMEOUT);
         for (int i = 0; i < kStages; ++i) {
           if (!((filled >> i) & 1u)) continue;
-          mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
+          if (leader) mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
+          if (EV > 0) mbar_wait_bounded(&zfull[i], (i < stage) ? phase : (phase ^ 1u));
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0; uint32_t phase = 0; int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
         const int m_blk = tile % P.num_m_blocks;
-        if (!tile_owned(P, m_blk)) continue;
+        if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         ++it;
-        if (!mbar_wait(&tm_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait<PAIR>(&tm_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         for (int kb = 0; kb < P.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * kABytes);
-          const uint32_t b_addr = smem_u32(sB + stage * kBBytes);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
           for (int k = 0; k < kBlockK / kUmmaK; ++k) {
             const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
             // N-major B: 16 K-rows of 128 B per step; 64-column groups 8 KB apart
             const uint64_t bdesc = smem_desc_sw128(b_addr + k * 2048, kBlockK * 128, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, kIdesc, (kb | k) != 0);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
+            else umma_bf16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR) umma_commit_pair_mc(&empty[stage], 0x3);
+          else umma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tm_full[acc]);
+        if constexpr (PAIR) umma_commit_pair_mc(&tm_full[acc], 0x3);
+        else umma_commit(&tm_full[acc]);
       }
       if (!ok) {
         *abort_flag = 1;
         raise_status(A.status, TWELL_ERR_TIMEOUT);
       }
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair_mc(drain, 0x1);
+      else umma_commit(drain);
       mbar_wait_bounded(drain, 0);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ slot producer (TMA)
+    if (TSLOT && lane == 0) {
+      const int E = A.E;
+      const uint32_t bytes = static_cast<uint32_t>(ring_entry);
+      int cnt = 0;
+      bool ok = true;
+      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
+        const int m_blk = tile % P.num_m_blocks;
+        if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
+        const int r0 = m_blk * TILE_M + row_base;
+        for (int t = 0; t < A.T; ++t, ++cnt) {
+          const int ring = cnt % kSlotRing;
+          const uint32_t ph = static_cast<uint32_t>(cnt / kSlotRing) & 1u;
+          if (!mbar_wait(&s_empty[ring], ph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&s_full[ring], bytes);
+          uint8_t *dst = sRing + ring * ring_entry;
+          tma_load_2d(dst, &tmap_sv, &s_full[ring], t * E, r0);
+          tma_load_2d(dst + ring_v, &tmap_si, &s_full[ring], (t * E) & ~15, r0);
+          tma_load_2d(dst + ring_v + ring_i, &tmap_sn, &s_full[ring], t & ~7, r0);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(A.status, TWELL_ERR_TIMEOUT);
+        for (int i = 0; i < kSlotRing && i < cnt; ++i)   // let issued copies land
+          mbar_wait_bounded(&s_full[i], static_cast<uint32_t>((cnt - 1 - ((cnt - 1 - i) % kSlotRing)) / kSlotRing) & 1u);
+      }
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = unit0; tile < num_tiles; tile += n_units) {
       const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
-      if (!tile_owned(P, m_blk)) continue;
+      if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       ++it;
-      if (!mbar_wait(&tm_full[acc], acc_phase, abort_flag)) {
+      if (!mbar_wait<PAIR>(&tm_full[acc], acc_phase, abort_flag)) {
         *abort_flag = 1;
         raise_status(A.status, TWELL_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
-      const int r = m_blk * kBlockM + row_in_tile;
+      const int r = m_blk * TILE_M + row_base + row_in_tile;
       const bool valid = r < A.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
       uint16_t *yr = P.y + static_cast<size_t>(r) * P.d + n_blk * kBN;
@@ -206,7 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tm_empty[acc]);
+      if (lane == 0) {   // accumulator free again (the MMAs are issued by the leader)
+        if constexpr (PAIR) mbar_arrive_cluster(map_to_cta(&tm_empty[acc], 0));
+        else mbar_arrive(&tm_empty[acc]);
+      }
     }
   } else if constexpr (EV > 0) {
     // ------------------------------------------------------------ A builders (fast)
@@ -221,16 +303,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_ovf = min(*A.n_ovf, A.cap);
     const uint32_t row_swz = static_cast<uint32_t>(row_in_tile & 7);
     int stage = 0; uint32_t phase = 0;
+    int scnt = 0;   // slot-ring records consumed so far (TSLOT)
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
       const int m_blk = tile % P.num_m_blocks;
-      if (!tile_owned(P, m_blk)) continue;
-      const int r = m_blk * kBlockM + row_in_tile;
+      if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
+      const int r = m_blk * TILE_M + row_base + row_in_tile;
       const bool valid = r < A.M;
       const size_t pair0 = static_cast<size_t>(valid ? r : 0) * Tn;
 
       // tile t's slot record of this row, straight into registers
       auto fetch = [&](int t, uint4 (&v)[EV], uint2 (&ix)[EV], int &n) {
+        if constexpr (TSLOT) return;                     // the ring path does its own reads
         if (valid && t < Tn) {
           const uint4 *gv = reinterpret_cast<const uint4 *>(A.vals + (pair0 + t) * E);
           const uint2 *gi = reinterpret_cast<const uint2 *>(A.idx + (pair0 + t) * E);
@@ -252,14 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb0 = 0; kb0 < P.num_kb && ok; kb0 += S) {
         const int nsteps = min(S, P.num_kb - kb0);
         const int stage0 = stage;
-        for (int j = 0; j < nsteps; ++j) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t *rowA = sA + stage * kABytes + row_in_tile * 128;
-          // Rows are 128 B apart, so lanes storing the same chunk index would all
-          // hit the same 4 banks; row-XOR chunk order makes the zeroing conflict-free.
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            reinterpret_cast<uint4 *>(rowA)[c ^ static_cast<int>(row_swz)] = make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < nsteps; ++j) {   // each step's A buffer, already zeroed by TMA
+          if (!mbar_wait(&zfull[stage], phase, abort_flag)) { ok = false; break; }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
@@ -267,14 +345,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t_last = (col0 + span - 1) >> lg_tw;
         for (int t = col0 >> lg_tw; t <= t_last; ++t) {   // 1 tile, or 2 when tile_w == 32
           if (t != cur_t) {                                // same for every thread of the CTA
-            if (cur_t < 0) {
-              fetch(t, vq, iq, n0);
-            } else {
+            if constexpr (TSLOT) {
+              // tile t's record waits in ring slot scnt % kSlotRing (filled by TMA)
+              const int ring = scnt % kSlotRing;
+              if (!mbar_wait(&s_full[ring], static_cast<uint32_t>(scnt / kSlotRing) & 1u, abort_flag)) {
+                ok = false;
+                break;
+              }
+              const uint8_t *base_r = sRing + ring * ring_entry;
+              const uint8_t *rv = base_r + row_in_tile * (2 * E);
+              const uint8_t *ri = base_r + ring_v + row_in_tile * P.slot_ib + ((t * E) & 15);
 #pragma unroll
-              for (int g = 0; g < EV; ++g) { vq[g] = vq1[g]; iq[g] = iq1[g]; }
-              n0 = n1;
+              for (int g = 0; g < EV; ++g) {
+                vq[g] = *reinterpret_cast<const uint4 *>(rv + 16 * g);
+                iq[g] = *reinterpret_cast<const uint2 *>(ri + 8 * g);
+              }
+              n0 = (valid && t < Tn)
+                       ? static_cast<int>(*reinterpret_cast<const uint16_t *>(
+                             base_r + ring_v + ring_i + row_in_tile * 16 + (t & 7) * 2))
+                       : 0;
+              // the previous slot's values are in registers by now: hand it back
+              if (scnt > 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[(scnt - 1) % kSlotRing]);
+              }
+              ++scnt;
+            } else {
+              if (cur_t < 0) {
+                fetch(t, vq, iq, n0);
+              } else {
+#pragma unroll
+                for (int g = 0; g < EV; ++g) { vq[g] = vq1[g]; iq[g] = iq1[g]; }
+                n0 = n1;
+              }
+              fetch(t + 1, vq1, iq1, n1);                  // one tile ahead; used next advance
             }
-            fetch(t + 1, vq1, iq1, n1);                    // one tile ahead; used next advance
             cur_t = t;
             ovf_k = (n0 > E) ? find_ovf(A.ovf_pos, n_ovf, static_cast<int>(pair0) + t) : -1;
           }
@@ -315,11 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0) {   // the MMA (leader CTA) may read these A rows now
           for (int j = 0; j < nsteps; ++j) {
             int sb = stage0 + j;
             if (sb >= kStages) sb -= kStages;
-            mbar_arrive(&full[sb]);
+            if constexpr (PAIR) mbar_arrive_cluster(map_to_cta(&full[sb], 0));
+            else mbar_arrive(&full[sb]);
           }
         }
       }
@@ -390,20 +496,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, 512);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, 512);
+    else tmem_dealloc(tmem_base, 512);
   }
 }
 
-// Per 128-token block: 1 when its density is at or above the crossover.
-__global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover, int32_t *blk_path) {
+// Per group of `rows` tokens (128, or 256 when the tensor-core path runs as CTA
+// pairs): 1 when its density is at or above the crossover.  The flag is written
+// for each 128-token block of the group so both down kernels read one array.
+__global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover, int rows,
+                                                    int32_t *blk_path) {
   const int blk = blockIdx.x;
-  const int r0 = blk * kBlockM;
-  const int rows = min(kBlockM, A.M - r0);
-  const long long n = static_cast<long long>(rows) * A.T;
+  const int r0 = blk * rows;
+  const int nr = min(rows, A.M - r0);
+  const long long n = static_cast<long long>(nr) * A.T;
   const uint16_t *base = A.nnz + static_cast<size_t>(r0) * A.T;
   unsigned long long sum = 0;
   for (long long i = threadIdx.x; i < n; i += blockDim.x) sum += __ldg(base + i);
@@ -415,27 +525,82 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    const double dens = static_cast<double>(red[0]) / (static_cast<double>(rows) * A.f);
-    blk_path[blk] = dens >= crossover ? 1 : 0;
+    const double dens = static_cast<double>(red[0]) / (static_cast<double>(nr) * A.f);
+    const int flag = dens >= crossover ? 1 : 0;
+    for (int b = r0 / kBlockM; b * kBlockM < r0 + nr; ++b) blk_path[b] = flag;
+  }
+}
+
+template <int EV, bool TSLOT, bool PAIR>
+cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUtensorMap &si,
+                        const CUtensorMap &sn, const DownParams &P, int num_sms, size_t smem,
+                        cudaStream_t s) {
+  auto kern = k_spmm_mma<EV, TSLOT, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int tiles = P.num_m_blocks * P.num_n_blocks;
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent static schedule: only as many pairs as can be resident at once
+    cfg.gridDim = dim3(num_sms & ~1, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms / 2;
+    int pairs = n < num_sms / 2 ? n : num_sms / 2;
+    if (pairs > tiles) pairs = tiles;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    return cudaLaunchKernelEx(&cfg, kern, mw, sv, si, sn, P);
+  } else {
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    kern<<<grid, kThreads, smem, s>>>(mw, sv, si, sn, P);
+    return cudaGetLastError();
   }
 }
 
 template <int EV>
-cudaError_t launch_down(const CUtensorMap &mw, const DownParams &P, int grid, size_t smem,
-                        cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(k_spmm_mma<EV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  k_spmm_mma<EV><<<grid, kThreads, smem, s>>>(mw, P);
-  return cudaGetLastError();
+cudaError_t launch_down_ev(bool tslot, bool pair, const CUtensorMap &mw, const CUtensorMap &sv,
+                           const CUtensorMap &si, const CUtensorMap &sn, const DownParams &P,
+                           int num_sms, size_t smem, cudaStream_t s) {
+  if constexpr (EV > 0) {
+    if (pair) {
+      return tslot ? launch_down<EV, true, true>(mw, sv, si, sn, P, num_sms, smem, s)
+                   : launch_down<EV, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+    }
+    if (tslot) return launch_down<EV, true, false>(mw, sv, si, sn, P, num_sms, smem, s);
+  }
+  return launch_down<EV, false, false>(mw, sv, si, sn, P, num_sms, smem, s);
 }
 
 }  // namespace
 
+// CTA-pair mode for this kernel is opt-in (TWELL_DOWN_CTA_PAIR=1): measured on
+// the 1.5B layer it is slower than one CTA per tile, because the pair's MMA
+// waits for the slower of two builder sets and the builders, not operand
+// bandwidth, bound this kernel.
+bool down_uses_pair(const TwellView &v) {
+  static int env = -1;
+  if (env < 0) {
+    const char *e = getenv("TWELL_DOWN_CTA_PAIR");
+    env = (e != nullptr && e[0] == '1') ? 1 : 0;
+  }
+  return env == 1 && v.E % 8 == 0 && v.E <= 64;
+}
+
 cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s) {
-  const int blocks = (v.M + kBlockM - 1) / kBlockM;
+  const int rows = down_uses_pair(v) ? 2 * kBlockM : kBlockM;
+  const int blocks = (v.M + rows - 1) / rows;
   if (blocks == 0) return cudaSuccess;
-  k_block_path<<<blocks, 256, 0, s>>>(v, crossover, blk_path);
+  k_block_path<<<blocks, 256, 0, s>>>(v, crossover, rows, blk_path);
   return cudaGetLastError();
 }
 
@@ -455,25 +620,43 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   P.num_kb = (v.f + kBlockK - 1) / kBlockK;
   P.blk_path = blk_path;
   const int ev = (v.E % 8 == 0 && v.E <= 64) ? v.E / 8 : 0;
-  const size_t fixed = 1024 + 256;
+  // Slot records by TMA: the row pitches of vals / idx / nnz must be multiples of
+  // 16 bytes and every box start 16-byte aligned (ell_w % 8 == 0, T % 8 == 0).
+  const int ib = (v.E % 16 == 0) ? v.E : v.E + 8;
+  bool tslot = ev > 0 && v.T % 8 == 0 && (static_cast<long long>(v.T) * v.E) % 16 == 0;
+  CUtensorMap sv = mw, si = mw, sn = mw;
+  if (tslot) {
+    const uint64_t te = static_cast<uint64_t>(v.T) * v.E;
+    tslot = encode_tensor_map_2d(&sv, v.vals, te, v.M, te * 2, v.E, kBlockM,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT16) == CUDA_SUCCESS &&
+            encode_tensor_map_2d(&si, v.idx, te, v.M, te, ib, kBlockM, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                 CU_TENSOR_MAP_DATA_TYPE_UINT8) == CUDA_SUCCESS &&
+            encode_tensor_map_2d(&sn, v.nnz, v.T, v.M, static_cast<uint64_t>(v.T) * 2, 8, kBlockM,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_UINT16) == CUDA_SUCCESS;
+  }
+  P.slot_ib = ib;
+  const bool pair = down_uses_pair(v);
+  const int tile_m = pair ? 2 * kBlockM : kBlockM;
+  P.num_m_blocks = (v.M + tile_m - 1) / tile_m;
+  const size_t b_stage = pair ? kBBytes / 2 : kBBytes;
+  const size_t ring = tslot ? static_cast<size_t>(kSlotRing) * kBlockM * (2 * v.E + ib + 16) : 0;
+  const size_t fixed = 1024 + 512 + ring;
   const size_t budget = 227 * 1024;
-  int stages = static_cast<int>((budget - fixed) / (kABytes + kBBytes));
+  int stages = static_cast<int>((budget - fixed) / (kABytes + b_stage));
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
   P.stages = stages;
-  const size_t smem = fixed + static_cast<size_t>(stages) * (kABytes + kBBytes);
-  const int tiles = P.num_m_blocks * P.num_n_blocks;
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const size_t smem = fixed + static_cast<size_t>(stages) * (kABytes + b_stage);
   switch (ev) {
-    case 1: return launch_down<1>(mw, P, grid, smem, s);
-    case 2: return launch_down<2>(mw, P, grid, smem, s);
-    case 3: return launch_down<3>(mw, P, grid, smem, s);
-    case 4: return launch_down<4>(mw, P, grid, smem, s);
-    case 5: return launch_down<5>(mw, P, grid, smem, s);
-    case 6: return launch_down<6>(mw, P, grid, smem, s);
-    case 7: return launch_down<7>(mw, P, grid, smem, s);
-    case 8: return launch_down<8>(mw, P, grid, smem, s);
-    default: return launch_down<0>(mw, P, grid, smem, s);
+    case 1: return launch_down_ev<1>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 2: return launch_down_ev<2>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 3: return launch_down_ev<3>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 4: return launch_down_ev<4>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 5: return launch_down_ev<5>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 6: return launch_down_ev<6>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 7: return launch_down_ev<7>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    case 8: return launch_down_ev<8>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
+    default: return launch_down_ev<0>(false, false, mw, sv, si, sn, P, num_sms, smem, s);
   }
 }
 

@@ -21,23 +21,31 @@
 // The two TMEM accumulators let the epilogue of tile i overlap the MMAs of
 // tile i+1.  Gated layers use N = 2*tile_w: gate rows then up rows of the same
 // hidden tile, so one accumulator holds g and u side by side.
+#include <cstdlib>
+
 #include "twell_device.cuh"
 
 namespace twell {
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kABytes = kBlockM * kBlockK * 2;   // 16 KB
 constexpr int kThreads = 192;
 
-template <int TW, bool GATED>
+// PAIR: a cluster of 2 CTAs computes a 256-token tile with M=256 MMAs
+// (tcgen05 cta_group::2); each CTA loads its 128 token rows and half of the
+// weight rows, so every SM moves half the operand bytes per FLOP.
+template <int TW, bool GATED, bool PAIR>
 struct UpCfg {
   static constexpr int N = GATED ? 2 * TW : 256;           // MMA N (accumulator columns)
   static constexpr int TILES_PER_ACC = GATED ? 1 : 256 / TW;
-  static constexpr int B_BYTES = N * kBlockK * 2;
-  static constexpr int STAGE_BYTES = kABytes + B_BYTES;
+  static constexpr int TILE_M = PAIR ? 2 * kBlockM : kBlockM;
+  static constexpr int B_ROWS = PAIR ? N / 2 : N;          // weight rows held by this CTA
+  static constexpr int B_BYTES = B_ROWS * kBlockK * 2;
+  static constexpr int STAGE_BYTES = kABytes + B_BYTES;    // per CTA
+  static constexpr int TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
   static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(kBlockM, N, 0, 0);
+  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, N, 0, 0);
 };
 
 struct UpParams {
@@ -60,11 +68,12 @@ __device__ __forceinline__ void load_bias8(const uint16_t *b, int col, float (&b
   for (int i = 0; i < 4; ++i) { bv[2 * i] = bf16lo_to_f32(w[i]); bv[2 * i + 1] = bf16hi_to_f32(w[i]); }
 }
 
-template <int TW, bool GATED>
+template <int TW, bool GATED, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     k_up_pack(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
               const __grid_constant__ CUtensorMap tmap_g, const UpParams P) {
-  using C = UpCfg<TW, GATED>;
+  using C = UpCfg<TW, GATED, PAIR>;
+  constexpr int kStages = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -73,11 +82,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sB = smem + kStages * kABytes;               // kStages x B_BYTES
   uint8_t *sSlots = sB + kStages * C::B_BYTES;          // 128 rows of slots
   const int E = P.out.E;
-  const int pitch_v = ((2 * E + 15) / 16) * 16 + 16;    // bf16 values (+16 B to spread banks)
-  const int pitch_i = ((E + 15) / 16) * 16;             // u8 indices
-  uint8_t *sVals = sSlots;
-  uint8_t *sIdx = sSlots + kBlockM * pitch_v;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sIdx + kBlockM * pitch_i);   // 2 KB aligned
+  // one 32-bit word per slot (bf16 value | in-tile index << 16); the row pitch is
+  // an odd number of words so lanes appending at equal counts hit distinct banks
+  const int pitch_w = E + 1 - (E & 1);
+  uint32_t *sSlotw = reinterpret_cast<uint32_t *>(sSlots);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(
+      sSlots + ((static_cast<size_t>(kBlockM) * pitch_w * 4 + 127) & ~static_cast<size_t>(127)));
   uint64_t *full = bars;
   uint64_t *empty = bars + kStages;
   uint64_t *tm_full = bars + 2 * kStages;
@@ -91,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], 4); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], PAIR ? 8 : 4); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -100,16 +110,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (GATED) tma_prefetch_desc(&tmap_g);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) { tmem_alloc_pair(tmem_slot, C::TMEM_COLS); tmem_relinquish_pair(); }
+    else { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_tiles = P.num_m_blocks * P.num_n_blocks;
   int32_t *status = P.out.status;
+  // work unit = one CTA (or one CTA pair) and its tile stride
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -117,19 +132,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0; uint32_t phase = 0;
       uint32_t filled = 0;   // bit i: stage i has been filled at least once
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
         const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
+        const int a_row = m_blk * C::TILE_M + static_cast<int>(rank) * kBlockM;
         for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          // the pair's bytes are all counted on the leader's barrier
+          if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
           filled |= 1u << stage;
-          tma_load_2d(sA + stage * kABytes, &tmap_x, &full[stage], kb * kBlockK, m_blk * kBlockM);
+          uint8_t *a_dst = sA + stage * kABytes;
           uint8_t *b_dst = sB + stage * C::B_BYTES;
-          if constexpr (GATED) {
-            tma_load_2d(b_dst, &tmap_g, &full[stage], kb * kBlockK, n_blk * TW);
-            tma_load_2d(b_dst + TW * 128, &tmap_w, &full[stage], kb * kBlockK, n_blk * TW);
+          if constexpr (PAIR) {
+            const uint32_t bar = map_to_cta(&full[stage], 0);
+            tma_load_2d_pair(a_dst, &tmap_x, bar, kb * kBlockK, a_row);
+            if constexpr (GATED)   // even CTA: gate rows, odd CTA: up rows of the hidden tile
+              tma_load_2d_pair(b_dst, rank == 0 ? &tmap_g : &tmap_w, bar, kb * kBlockK, n_blk * TW);
+            else
+              tma_load_2d_pair(b_dst, &tmap_w, bar, kb * kBlockK, n_blk * 256 + static_cast<int>(rank) * C::B_ROWS);
           } else {
-            tma_load_2d(b_dst, &tmap_w, &full[stage], kb * kBlockK, n_blk * 256);
+            tma_load_2d(a_dst, &tmap_x, &full[stage], kb * kBlockK, a_row);
+            if constexpr (GATED) {
+              tma_load_2d(b_dst, &tmap_g, &full[stage], kb * kBlockK, n_blk * TW);
+              tma_load_2d(b_dst + TW * 128, &tmap_w, &full[stage], kb * kBlockK, n_blk * TW);
+            } else {
+              tma_load_2d(b_dst, &tmap_w, &full[stage], kb * kBlockK, n_blk * 256);
+            }
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -140,27 +167,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Let issued copies land before the CTA's shared memory goes away: the
         // most recent fill of stage i used phase parity `phase` for stages below
         // the ring position and `phase ^ 1` for the others.
-        for (int i = 0; i < kStages; ++i) {
-          if (!((filled >> i) & 1u)) continue;
-          const uint32_t par = (i < stage) ? phase : (phase ^ 1u);
-          mbar_wait_bounded(&full[i], par);
+        if (leader) {   // (the odd CTA's copies are counted on the leader's barriers)
+          for (int i = 0; i < kStages; ++i) {
+            if (!((filled >> i) & 1u)) continue;
+            const uint32_t par = (i < stage) ? phase : (phase ^ 1u);
+            mbar_wait_bounded(&full[i], par);
+          }
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0; uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++it) {
+      for (int tile = unit0; tile < num_tiles && ok; tile += n_units, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait(&tm_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait<PAIR>(&tm_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::N);
         for (int kb = 0; kb < P.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * kABytes);
           const uint32_t b_addr = smem_u32(sB + stage * C::B_BYTES);
@@ -168,41 +197,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < kBlockK / kUmmaK; ++k) {
             const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_addr + k * 32, 16, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, C::IDESC, (kb | k) != 0);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, adesc, bdesc, C::IDESC, (kb | k) != 0);
+            else umma_bf16(d_tmem, adesc, bdesc, C::IDESC, (kb | k) != 0);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR) umma_commit_pair_mc(&empty[stage], 0x3);   // frees the stage in both CTAs
+          else umma_commit(&empty[stage]);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tm_full[acc]);
+        if constexpr (PAIR) umma_commit_pair_mc(&tm_full[acc], 0x3);
+        else umma_commit(&tm_full[acc]);
       }
       if (!ok) {
         *abort_flag = 1;
         raise_status(status, TWELL_ERR_TIMEOUT);
       }
       // all issued MMAs must finish before TMEM is released
-      umma_commit(drain);
+      if constexpr (PAIR) umma_commit_pair_mc(drain, 0x1);
+      else umma_commit(drain);
       mbar_wait_bounded(drain, 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const int row_in_tile = q * 32 + lane;
-    uint16_t *my_vals = reinterpret_cast<uint16_t *>(sVals + row_in_tile * pitch_v);
-    uint8_t *my_idx = sIdx + row_in_tile * pitch_i;
+    uint32_t *my_slots = sSlotw + row_in_tile * pitch_w;
     const PackTarget &O = P.out;
     int it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+    for (int tile = unit0; tile < num_tiles; tile += n_units, ++it) {
       const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(&tm_full[acc], acc_phase, abort_flag)) {
+      if (!mbar_wait<PAIR>(&tm_full[acc], acc_phase, abort_flag)) {
         *abort_flag = 1;
         raise_status(status, TWELL_ERR_TIMEOUT);
         break;
       }
       tc_fence_after();
-      const int r = m_blk * kBlockM + row_in_tile;
+      const int r = m_blk * C::TILE_M + static_cast<int>(rank) * kBlockM + row_in_tile;
       const bool valid = r < P.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::N);
 
@@ -248,9 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               if constexpr (GATED) v = __fmul_rn(v, __uint_as_float(g[j]));
               const uint32_t hb = bf16_bits_rn(v);
               const bool nz = (hb & 0x7FFFu) != 0;
-              if (nz && cnt < E) {
-                my_vals[cnt] = static_cast<uint16_t>(hb);
-                my_idx[cnt] = static_cast<uint8_t>(c * 32 + j);
+              const bool put = nz && cnt < E;
+              if (__any_sync(0xFFFFFFFFu, put)) {   // no store issued for all-zero columns
+                if (put) my_slots[cnt] = hb | (static_cast<uint32_t>(c * 32 + j) << 16);
               }
               cnt += nz ? 1 : 0;
             }
@@ -262,32 +294,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint16_t *gv = O.vals + pair * E;
           uint8_t *gi = O.idx + pair * E;
           if ((E & 7) == 0) {
-            for (int s = 0; s < E; s += 8) {
-              uint4 w = *reinterpret_cast<const uint4 *>(my_vals + s);
-              uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+            for (int s = 0; s < E; s += 8) {   // slots >= cnt are padding: (+0, 0)
+              uint32_t w[8];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {   // slots >= cnt are padding: (+0, 0)
-                const int s0 = s + 2 * i;
-                if (s0 >= cnt) ww[i] = 0;
-                else if (s0 + 1 >= cnt) ww[i] &= 0x0000FFFFu;
-              }
-              *reinterpret_cast<uint4 *>(gv + s) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
-              uint2 iw = *reinterpret_cast<const uint2 *>(my_idx + s);
-              uint32_t ib[2] = {iw.x, iw.y};
-#pragma unroll
-              for (int i = 0; i < 2; ++i) {
-                uint32_t m = 0;
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb)
-                  if (s + 4 * i + bb < cnt) m |= 0xFFu << (8 * bb);
-                ib[i] &= m;
-              }
-              *reinterpret_cast<uint2 *>(gi + s) = make_uint2(ib[0], ib[1]);
+              for (int i = 0; i < 8; ++i) w[i] = (s + i < cnt) ? my_slots[s + i] : 0u;
+              *reinterpret_cast<uint4 *>(gv + s) =
+                  make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                             __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+              *reinterpret_cast<uint2 *>(gi + s) =
+                  make_uint2(__byte_perm(__byte_perm(w[0], w[1], 0x6262), __byte_perm(w[2], w[3], 0x6262), 0x5410),
+                             __byte_perm(__byte_perm(w[4], w[5], 0x6262), __byte_perm(w[6], w[7], 0x6262), 0x5410));
             }
           } else {
             for (int s = 0; s < E; ++s) {
-              gv[s] = (s < cnt) ? my_vals[s] : static_cast<uint16_t>(0);
-              gi[s] = (s < cnt) ? my_idx[s] : static_cast<uint8_t>(0);
+              const uint32_t w = (s < cnt) ? my_slots[s] : 0u;
+              gv[s] = static_cast<uint16_t>(w & 0xFFFFu);
+              gi[s] = static_cast<uint8_t>(w >> 16);
             }
           }
         }
@@ -337,35 +359,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tm_empty[acc]);
+      if (lane == 0) {   // the accumulator may be overwritten (MMAs are issued by the leader)
+        if constexpr (PAIR) mbar_arrive_cluster(map_to_cta(&tm_empty[acc], 0));
+        else mbar_arrive(&tm_empty[acc]);
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
-template <int TW, bool GATED>
+template <int TW, bool GATED, bool PAIR>
 size_t up_smem_bytes(int E) {
-  using C = UpCfg<TW, GATED>;
-  const int pitch_v = ((2 * E + 15) / 16) * 16 + 16;
-  const int pitch_i = ((E + 15) / 16) * 16;
-  return 1024 + kStages * (kABytes + C::B_BYTES) + kBlockM * (pitch_v + pitch_i) + 64 + 256;
+  using C = UpCfg<TW, GATED, PAIR>;
+  const int pitch_w = E + 1 - (E & 1);
+  const size_t slots = (static_cast<size_t>(kBlockM) * pitch_w * 4 + 127) & ~static_cast<size_t>(127);
+  return 1024 + C::STAGES * (kABytes + C::B_BYTES) + slots + 256;
 }
 
-template <int TW, bool GATED>
+// CTA pairing is on unless TWELL_UP_CTA_PAIR=0 (a tuning / comparison knob).
+bool use_cta_pair() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("TWELL_UP_CTA_PAIR");
+    v = (e != nullptr && e[0] == '0') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+template <int TW, bool GATED, bool PAIR>
 cudaError_t launch_up_impl(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s) {
-  using C = UpCfg<TW, GATED>;
+  using C = UpCfg<TW, GATED, PAIR>;
   CUtensorMap mx, mw, mg;
   if (encode_tensor_map_2d(&mx, a.x, a.d, a.M, static_cast<uint64_t>(a.d) * 2, kBlockK, kBlockM,
                            CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  const uint32_t w_rows = GATED ? TW : 256;
+  const uint32_t w_rows = GATED ? TW : C::B_ROWS;
   if (encode_tensor_map_2d(&mw, a.w_up, a.d, a.f, static_cast<uint64_t>(a.d) * 2, kBlockK, w_rows,
                            CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -379,19 +415,54 @@ cudaError_t launch_up_impl(const UpArgs &a, const PackTarget &t, int num_sms, cu
   UpParams P;
   P.b = a.b;
   P.M = a.M; P.d = a.d; P.f = a.f;
-  P.num_m_blocks = (a.M + kBlockM - 1) / kBlockM;
+  P.num_m_blocks = (a.M + C::TILE_M - 1) / C::TILE_M;
   P.num_n_blocks = GATED ? t.T : (a.f + 255) / 256;
   P.num_kb = a.d / kBlockK;
   P.z_debug = a.z_debug;
   P.out = t;
-  const size_t smem = up_smem_bytes<TW, GATED>(t.E);
-  cudaError_t e = cudaFuncSetAttribute(k_up_pack<TW, GATED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = up_smem_bytes<TW, GATED, PAIR>(t.E);
+  cudaError_t e = cudaFuncSetAttribute(k_up_pack<TW, GATED, PAIR>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = P.num_m_blocks * P.num_n_blocks;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  k_up_pack<TW, GATED><<<grid, kThreads, smem, s>>>(mx, mw, mg, P);
-  return cudaGetLastError();
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // The schedule is persistent and static, so launch only as many pairs as can
+    // be resident at once (SM pairing depends on the GPU's cluster layout).
+    static int max_pairs = 0;
+    if (max_pairs == 0) {
+      cfg.gridDim = dim3(num_sms & ~1, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_up_pack<TW, GATED, true>, &cfg) != cudaSuccess || n < 1)
+        n = num_sms / 2;
+      max_pairs = n;
+    }
+    int pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
+    if (pairs > tiles) pairs = tiles;
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    return cudaLaunchKernelEx(&cfg, k_up_pack<TW, GATED, true>, mx, mw, mg, P);
+  } else {
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    k_up_pack<TW, GATED, false><<<grid, kThreads, smem, s>>>(mx, mw, mg, P);
+    return cudaGetLastError();
+  }
+}
+
+template <int TW, bool GATED>
+cudaError_t launch_up_sel(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s) {
+  return use_cta_pair() ? launch_up_impl<TW, GATED, true>(a, t, num_sms, s)
+                        : launch_up_impl<TW, GATED, false>(a, t, num_sms, s);
 }
 
 }  // namespace
@@ -400,10 +471,10 @@ cudaError_t launch_up_pack(const UpArgs &a, const PackTarget &t, int num_sms, cu
   if (a.M == 0) return cudaSuccess;
   const bool gated = a.w_gate != nullptr;
   switch (t.tw) {
-    case 32: return gated ? launch_up_impl<32, true>(a, t, num_sms, s) : launch_up_impl<32, false>(a, t, num_sms, s);
-    case 64: return gated ? launch_up_impl<64, true>(a, t, num_sms, s) : launch_up_impl<64, false>(a, t, num_sms, s);
-    case 128: return gated ? launch_up_impl<128, true>(a, t, num_sms, s) : launch_up_impl<128, false>(a, t, num_sms, s);
-    case 256: return gated ? cudaErrorNotSupported : launch_up_impl<256, false>(a, t, num_sms, s);
+    case 32: return gated ? launch_up_sel<32, true>(a, t, num_sms, s) : launch_up_sel<32, false>(a, t, num_sms, s);
+    case 64: return gated ? launch_up_sel<64, true>(a, t, num_sms, s) : launch_up_sel<64, false>(a, t, num_sms, s);
+    case 128: return gated ? launch_up_sel<128, true>(a, t, num_sms, s) : launch_up_sel<128, false>(a, t, num_sms, s);
+    case 256: return gated ? cudaErrorNotSupported : launch_up_sel<256, false>(a, t, num_sms, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -200,14 +200,14 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                               uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
-                              CUtensorMapSwizzle swizzle) {
+                              CUtensorMapSwizzle swizzle, CUtensorMapDataType dtype) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
   const cuuint64_t dims[2] = {inner, outer};
   const cuuint64_t strides[1] = {row_pitch_bytes};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t elem_strides[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+  return fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box,
             elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }

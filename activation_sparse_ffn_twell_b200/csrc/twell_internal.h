@@ -101,6 +101,7 @@ constexpr float kDownCrossoverDensity = 0.02f;
 // library loads on machines without a driver).
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                               uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
-                              CUtensorMapSwizzle swizzle);
+                              CUtensorMapSwizzle swizzle,
+                              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 
 }  // namespace twell
