@@ -33,7 +33,10 @@ constexpr int kMaxStages = 6;
 constexpr int kBN = 256;                        // y columns per tile
 constexpr int kABytes = kBlockM * kBlockK * 2;  // 16 KB
 constexpr int kBBytes = kBlockK * kBN * 2;      // 32 KB (4 boxes of 64 x 64)
-constexpr int kThreads = 352;
+// warps: 0 TMA (W_down), 1 MMA, 2..5 epilogue, 6..13 A builders (two per token
+// row on the fast path), 14 slot producer
+constexpr int kThreads = 480;
+constexpr int kSlotWarp = 14;
 constexpr int kSlotRing = 4;                    // slot-record ring depth (hidden tiles)
 
 // Source of the per-stage A clear: the fast builders only write nonzeros, the
@@ -107,9 +110,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const TwellView &A = P.A;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], 1 + (PAIR ? 8 : 4)); mbar_init(&empty[i], 1); }
+    constexpr int kBuildWarps = EV > 0 ? 8 : 4;
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 1 + (PAIR ? 2 : 1) * kBuildWarps);
+      mbar_init(&empty[i], 1);
+    }
     for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], PAIR ? 8 : 4); }
-    for (int i = 0; i < kSlotRing; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4); }
+    for (int i = 0; i < kSlotRing; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8); }
     for (int i = 0; i < kStages; ++i) mbar_init(&zfull[i], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -215,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       else umma_commit(drain);
       mbar_wait_bounded(drain, 0);
     }
-  } else if (warp == 10) {
+  } else if (warp == kSlotWarp) {
     // ------------------------------------------------------------ slot producer (TMA)
     if (TSLOT && lane == 0) {
       const int E = A.E;
@@ -297,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // with independent 16-byte stores and every slot is written once with a
     // predicated 2-byte store -- a fully unrolled, dependency-free sequence.
     constexpr int E = 8 * EV;
-    const int row_in_tile = (warp - 6) * 32 + lane;
+    // two threads per token row: `half` takes the slots of its parity
+    const int row_in_tile = ((warp - 6) & 3) * 32 + lane;
+    const int half = (warp - 6) >> 2;
     const int tw = A.tw, Tn = A.T;
     const int lg_tw = 31 - __clz(tw);
     const int n_ovf = min(*A.n_ovf, A.cap);
@@ -386,28 +395,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!valid || t >= Tn || n0 == 0) continue;
           const int base = (t << lg_tw) - col0;           // group column of in-tile index 0
           if (n0 <= E) {
+            const uint32_t vsh = 16u * static_cast<uint32_t>(half);   // value half of each word
 #pragma unroll
             for (int g = 0; g < EV; ++g) {
               const uint32_t vw[4] = {vq[g].x, vq[g].y, vq[g].z, vq[g].w};
               const uint32_t iw[2] = {iq[g].x, iq[g].y};
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int sl = 8 * g + k;
-                const uint32_t col = static_cast<uint32_t>(base + static_cast<int>((iw[k >> 2] >> (8 * (k & 3))) & 0xFFu));
+              for (int k2 = 0; k2 < 4; ++k2) {   // slot 8g + 2*k2 + half
+                const int sl = 8 * g + 2 * k2 + half;
+                const uint32_t ib = (iw[k2 >> 1] >> (16u * (k2 & 1) + 8u * static_cast<uint32_t>(half))) & 0xFFu;
+                const uint32_t col = static_cast<uint32_t>(base + static_cast<int>(ib));
                 if (sl < n0 && col < static_cast<uint32_t>(span)) {
                   int sb = stage0 + static_cast<int>(col >> 6);   // step buffer of this column
                   if (sb >= kStages) sb -= kStages;
                   const uint32_t c = col & 63u;
                   const uint32_t off = (((c >> 3) ^ row_swz) << 4) + ((c & 7u) << 1);
                   *reinterpret_cast<uint16_t *>(sA + sb * kABytes + row_in_tile * 128 + off) =
-                      static_cast<uint16_t>((k & 1) ? (vw[k >> 1] >> 16) : (vw[k >> 1] & 0xFFFFu));
+                      static_cast<uint16_t>((vw[k2] >> vsh) & 0xFFFFu);
                 }
               }
             }
           } else if (ovf_k >= 0) {                        // dense backup segment
             // group columns c with in-tile index c - base inside [0, tile_w)
             const int lo = max(0, base), hi = min(span, base + tw);
-            for (int c = lo; c < hi; c += 8) {
+            for (int c = lo + 8 * half; c < hi; c += 16) {   // this thread's 16-B chunks
               const uint4 q = __ldg(reinterpret_cast<const uint4 *>(
                   A.ovf_dense + static_cast<size_t>(ovf_k) * tw + (c - base)));
               int sb = stage0 + (c >> 6);
@@ -434,8 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
       raise_status(A.status, TWELL_ERR_TIMEOUT);
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------ A builders (general)
+    // one thread per token row (warps 10..13 idle on this path)
     const int row_in_tile = (warp - 6) * 32 + lane;
     const int n_ovf = min(*A.n_ovf, A.cap);
     int stage = 0; uint32_t phase = 0;
