@@ -15,17 +15,6 @@
 namespace twell {
 namespace {
 
-__device__ __forceinline__ int find_ovf(const int32_t *pos, int n, int key) {
-  int lo = 0, hi = n - 1;
-  while (lo <= hi) {
-    const int mid = (lo + hi) >> 1;
-    const int v = __ldg(pos + mid);
-    if (v == key) return mid;
-    if (v < key) lo = mid + 1; else hi = mid - 1;
-  }
-  return -1;
-}
-
 template <int NCH>
 __device__ __forceinline__ void fma_row(float (&acc)[NCH][8], const uint16_t *wrow, int col_base,
                                         int d, float v) {
@@ -71,6 +60,7 @@ __global__ void __launch_bounds__(256) k_spmm_gather(TwellView A, const uint16_t
       for (int i = 0; i < 8; ++i) acc[ch][i] = 0.f;
 
     const size_t row_pair0 = static_cast<size_t>(r) * A.T;
+    int ovf_base = -1, ovf_seen = 0;
     for (int t0 = 0; t0 < A.T; t0 += 32) {
       const int tt = t0 + lane;
       const int my_n = (tt < A.T) ? static_cast<int>(__ldg(A.nnz + row_pair0 + tt)) : 0;
@@ -96,8 +86,10 @@ __global__ void __launch_bounds__(256) k_spmm_gather(TwellView A, const uint16_t
             }
           }
         } else {
-          const int k = find_ovf(A.ovf_pos, n_ovf, r * A.T + t);
-          if (k < 0) continue;   // capacity exhausted: status already raised, y undefined
+          // this token's backup entries are consecutive: search once, then walk
+          if (ovf_base < 0) ovf_base = ovf_lower_bound(A.ovf_pos, n_ovf, r * A.T);
+          const int k = ovf_base + ovf_seen++;
+          if (k >= n_ovf) continue;   // capacity exhausted: status already raised, y undefined
           const uint16_t *seg = A.ovf_dense + static_cast<size_t>(k) * A.tw;
           for (int j0 = 0; j0 < A.tw; j0 += 32) {
             const uint32_t sv = __ldg(seg + j0 + lane);

@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
 
-      int cur_t = -1, n0 = 0, n1 = 0, ovf_k = -1;
+      int cur_t = -1, n0 = 0, n1 = 0, ovf_k = -1, ovf_base = -1, ovf_seen = 0;
       uint4 vq[EV], vq1[EV];
       uint2 iq[EV], iq1[EV];
       // K-steps are claimed in groups of S (all steps of one hidden tile when
@@ -390,7 +390,15 @@ __global__ void __launch_bounds__(kThreads, 1)
               fetch(t + 1, vq1, iq1, n1);                  // one tile ahead; used next advance
             }
             cur_t = t;
-            ovf_k = (n0 > E) ? find_ovf(A.ovf_pos, n_ovf, static_cast<int>(pair0) + t) : -1;
+            // backup entry of an overflowing pair: this token's run of entries
+            // starts at ovf_base (found once per token), the k-th overflow tile
+            // of the row is entry ovf_base + k
+            ovf_k = -1;
+            if (n0 > E) {
+              if (ovf_base < 0) ovf_base = ovf_lower_bound(A.ovf_pos, n_ovf, static_cast<int>(pair0));
+              ovf_k = ovf_base + ovf_seen++;
+              if (ovf_k >= n_ovf) ovf_k = -1;   // capacity exhausted: y is undefined
+            }
           }
           if (!valid || t >= Tn || n0 == 0) continue;
           const int base = (t << lg_tw) - col0;           // group column of in-tile index 0
@@ -419,13 +427,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             // group columns c with in-tile index c - base inside [0, tile_w)
             const int lo = max(0, base), hi = min(span, base + tw);
             for (int c = lo + 8 * half; c < hi; c += 16) {   // this thread's 16-B chunks
-              const uint4 q = __ldg(reinterpret_cast<const uint4 *>(
-                  A.ovf_dense + static_cast<size_t>(ovf_k) * tw + (c - base)));
+              const uint16_t *src = A.ovf_dense + static_cast<size_t>(ovf_k) * tw + (c - base);
               int sb = stage0 + (c >> 6);
               if (sb >= kStages) sb -= kStages;
               const uint32_t cc = static_cast<uint32_t>(c & 63);
-              *reinterpret_cast<uint4 *>(sA + sb * kABytes + row_in_tile * 128 +
-                                         (((cc >> 3) ^ row_swz) << 4)) = q;
+              uint8_t *dst = sA + sb * kABytes + row_in_tile * 128 + (((cc >> 3) ^ row_swz) << 4);
+              if constexpr (!PAIR) {
+                // async-proxy copy counted on the stage's full barrier: no thread
+                // waits for it, and the MMA sees it through that barrier (posted
+                // before this warp's arrive, so the phase cannot complete early)
+                mbar_expect_tx(&full[sb], 16);
+                bulk_load(dst, src, 16, &full[sb]);
+              } else {
+                *reinterpret_cast<uint4 *>(dst) = __ldg(reinterpret_cast<const uint4 *>(src));
+              }
             }
           }
         }

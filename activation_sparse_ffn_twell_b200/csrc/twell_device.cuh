@@ -43,6 +43,18 @@ __device__ __forceinline__ void raise_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// First index of the ascending backup position list `pos[0..n)` whose value is
+// >= key (n if none).  A token's overflowing pairs are consecutive in the list
+// (positions r*T .. r*T+T-1), so consumers search once per token and then walk.
+__device__ __forceinline__ int ovf_lower_bound(const int32_t *pos, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(pos + mid) < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -61,6 +73,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
+               : "memory");
+}
+
+// Add `bytes` to the barrier's expected transaction count without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
 

@@ -95,7 +95,7 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
 
 // Density (nonzeros / (rows * d_ff)) of a 128-token block at or above which the
 // AUTO down-projection uses the tensor-core path.  Chosen from measurement.
-constexpr float kDownCrossoverDensity = 0.02f;
+constexpr float kDownCrossoverDensity = 0.006f;
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved at run time so the
 // library loads on machines without a driver).

@@ -131,9 +131,23 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------
-def _workload(density, M, seed):
+WORKLOADS = ("relu_15b", "gated_2b", "heavy_tail", "decode32", "decode128", "decode256", "tiny")
+
+
+def _workload(density, M, seed, name="relu_15b"):
+    """The synthetic layer for `name` (default: the 1.5B-scale ReLU layer)."""
     import twell_synth as S
-    return S.relu_15b(density=density, M=M, seed=seed)
+    if name == "relu_15b":
+        return S.relu_15b(density=density, M=M, seed=seed)
+    if name == "gated_2b":
+        return S.gated_2b(density=density, seed=seed)
+    if name == "heavy_tail":
+        return S.heavy_tail(seed=seed)
+    if name.startswith("decode"):
+        return S.decode(M=int(name[len("decode"):]), seed=seed)
+    if name == "tiny":
+        return S.tiny_relu(seed)
+    raise SystemExit(f"unknown workload {name}")
 
 
 def _roofline_layer(L, nnz_total, touched_rows, peaks):
@@ -163,8 +177,9 @@ def run_ours(args):
         import numpy as np
         return None if bits is None else torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    L = _workload(args.density, args.M, seed=args.seed + rank)   # own token batch per rank
+    L = _workload(args.density, args.M, args.seed + rank, args.workload)   # own batch per rank
     x, wu, b, wd = to_dev(L.x), to_dev(L.w_up), to_dev(L.b), to_dev(L.w_down)
+    wg = to_dev(L.w_gate)
     M, d, f, tw, E = L.M, L.d_model, L.d_ff, L.tile_w, L.ell_w
     T_tiles = f // tw
     a = T.TwELL.allocate(M, f, tw, E, T.default_ovf_capacity(M, T_tiles), device=dev)
@@ -173,7 +188,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        T.twell_up_pack(x, wu, b, tile_w=tw, ell_w=E, out=a)
+        T.twell_up_pack(x, wu, b, wg, tile_w=tw, ell_w=E, out=a)
         T.twell_spmm(a, wd, mode=args.mode, y=y)
 
     for _ in range(args.warmup):
@@ -200,7 +215,7 @@ def run_ours(args):
             flush.zero_()                      # evict L2 between steps (inputs < 126 MB)
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            T.twell_up_pack(x, wu, b, tile_w=tw, ell_w=E, out=a)
+            T.twell_up_pack(x, wu, b, wg, tile_w=tw, ell_w=E, out=a)
             e1.record(stream)
             T.twell_spmm(a, wd, mode=args.mode, y=y)
             e2.record(stream)
@@ -222,7 +237,7 @@ def run_ours(args):
     # Per-phase rooflines.  Up: 2*M*d*f FLOP on the tensor pipe.  Down: the
     # algorithmic work is 2*nnz*d FLOP; the tensor-core path executes the dense
     # 2*M*d*f on h tiles rebuilt from TwELL (reported as executed_tflops).
-    up_flop = 2.0 * M * d * f
+    up_flop = 2.0 * M * d * f * (2 if L.gated else 1)
     down_flop = 2.0 * nnz_total * d
     phases = {
         "up": {"kernel": "k_up_pack (fused up-GEMM + ReLU + TwELL pack, CTA pairs)",
@@ -233,7 +248,7 @@ def run_ours(args):
                            if args.mode != "gather" else "k_spmm_gather",
                  "ms": down_s * 1e3, "achieved": down_flop / down_s / 1e12, "unit": "TFLOP/s",
                  "frac": down_flop / down_s / 1e12 / peaks["tc_tflops"],
-                 "executed_tflops": up_flop / down_s / 1e12,
+                 "executed_tflops": 2.0 * M * d * f / down_s / 1e12,
                  "traffic": _ncu_traffic("k_spmm_mma.cu", f"relu_15b_rho{args.density:g}")},
     }
     dom = max(phases, key=lambda k: phases[k]["ms"])
@@ -243,9 +258,10 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1/fan_in) weights, bias for target density)",
-        "config": {"workload": "relu_ffn_layer_1.5b", "M": M, "d_model": d, "d_ff": f,
-                   "target_density": args.density, "measured_density": density,
-                   "tile_w": tw, "ell_w": E, "gated": False, "down_mode": args.mode,
+        "config": {"workload": {"relu_15b": "relu_ffn_layer_1.5b"}.get(args.workload, args.workload),
+                   "M": M, "d_model": d, "d_ff": f,
+                   "target_density": L.target_density, "measured_density": density,
+                   "tile_w": tw, "ell_w": E, "gated": bool(L.gated), "down_mode": args.mode,
                    "n_ovf": n_ovf, "l2": "flushed: 256 MiB write between timed steps",
                    "parallelism": f"token-sharded x{world} (weights replicated, no collective)"},
         "roofline": {"bound": "tensor", "kernel": P_["kernel"], "phase": dom,
@@ -265,12 +281,15 @@ def run_ours(args):
     result["clocks"] = clk.summary()
 
     if not args.quick:
-        result["dense_ffn"] = _dense_baseline(x, wu, b, wd, args, flush, stream, dev)
+        result["dense_ffn"] = _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg)
         result["e2e"] = _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world)
         if args.sweep:
             result["density_sweep"] = _sweep(T, args, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = _cpu_baseline(L, seconds=args.cpu_seconds)
+    if args.workload != "relu_15b":
+        result["note"] = ("extra workload (not the headline configuration); "
+                          "vs_baseline and the phase traffic refer to the 1.5B layer")
     if rank == 0:
         print(json.dumps(result), flush=True)
     del a
@@ -304,13 +323,16 @@ def _kernels_per_step(mode):
     return 3 + (3 if mode == "auto" else 1)
 
 
-def _dense_baseline(x, wu, b, wd, args, flush, stream, dev):
+def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):
     """Same-shape dense bf16 FFN through cuBLAS (torch.matmul), same run, same timing."""
     import torch
     import torch.nn.functional as F
 
     def dense():
-        h = torch.relu(F.linear(x, wu, b))
+        if wg is not None:   # gated: ReLU(x W_g^T + b) * (x W_u^T)
+            h = torch.relu(F.linear(x, wg, b)) * F.linear(x, wu)
+        else:
+            h = torch.relu(F.linear(x, wu, b))
         return torch.matmul(h, wd)
     for _ in range(max(3, args.warmup)):
         dense()
@@ -337,16 +359,19 @@ def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
     xh = torch.from_numpy(L.x.view(np.int16)).view(torch.bfloat16).pin_memory()
     yh = torch.empty((L.M, L.d_model), dtype=torch.bfloat16).pin_memory()
     xd = torch.empty_like(x)
+    wg = None if L.w_gate is None else torch.from_numpy(L.w_gate.view(np.int16)).view(torch.bfloat16).to(dev)
     for _ in range(3):
         xd.copy_(xh, non_blocking=True)
-        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=args.mode, out=a, y=y)
+        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg, mode=args.mode,
+                            out=a, y=y)
         yh.copy_(y, non_blocking=True)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         xd.copy_(xh, non_blocking=True)
-        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=args.mode, out=a, y=y)
+        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg, mode=args.mode,
+                            out=a, y=y)
         yh.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
@@ -431,7 +456,7 @@ def _cpu_baseline(L, seconds=10.0, sample_tokens=256):
     while True:
         r0 = (reps * sample_tokens) % L.M
         rows = slice(r0, r0 + sample_tokens)
-        O.ffn_forward(L.x[rows], L.w_up, L.b, L.w_down, L.tile_w, L.ell_w)
+        O.ffn_forward(L.x[rows], L.w_up, L.b, L.w_down, L.tile_w, L.ell_w, L.w_gate)
         done += min(sample_tokens, L.M - r0)
         reps += 1
         el = time.perf_counter() - t0
@@ -480,6 +505,8 @@ def main():
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--mode", default="auto", choices=["auto", "gather", "mma"])
+    ap.add_argument("--workload", default="relu_15b", choices=WORKLOADS,
+                    help="default: the 1.5B-scale layer the headline metric is quoted on")
     ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")
     ap.add_argument("--quick", action="store_true", help="skip dense/e2e legs (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
