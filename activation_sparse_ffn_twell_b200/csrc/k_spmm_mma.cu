@@ -37,7 +37,7 @@ constexpr int kBBytes = kBlockK * kBN * 2;      // 32 KB (4 boxes of 64 x 64)
 // row on the fast path), 14 slot producer
 constexpr int kThreads = 480;
 constexpr int kSlotWarp = 14;
-constexpr int kSlotRing = 4;                    // slot-record ring depth (hidden tiles)
+constexpr int kSlotRing = 4;                    // max slot-record ring depth (hidden tiles)
 
 // Source of the per-stage A clear: the fast builders only write nonzeros, the
 // TMA engine zeroes the stage first (a bulk copy from this never-written array),
@@ -51,6 +51,7 @@ struct DownParams {
   int num_m_blocks, num_n_blocks, num_kb;
   int stages;                // pipeline depth (<= kMaxStages), set from shared-memory budget
   int slot_ib;               // bytes of the index box per row (covers ell_w indices)
+  int ring;                  // slot-record ring depth (2..kSlotRing)
   const int32_t *blk_path;   // NULL, or per 128-token block: 1 = this path owns it
 };
 
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sRing = reinterpret_cast<uint8_t *>(bars) + 512;
   const int ring_v = kBlockM * 2 * P.A.E, ring_i = kBlockM * P.slot_ib;
   const int ring_entry = ring_v + ring_i + kBlockM * 16;
+  const int kRing = P.ring;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -234,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         const int r0 = m_blk * TILE_M + row_base;
         for (int t = 0; t < A.T; ++t, ++cnt) {
-          const int ring = cnt % kSlotRing;
-          const uint32_t ph = static_cast<uint32_t>(cnt / kSlotRing) & 1u;
+          const int ring = cnt % kRing;
+          const uint32_t ph = static_cast<uint32_t>(cnt / kRing) & 1u;
           if (!mbar_wait(&s_empty[ring], ph ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&s_full[ring], bytes);
           uint8_t *dst = sRing + ring * ring_entry;
@@ -247,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         *abort_flag = 1;
         raise_status(A.status, TWELL_ERR_TIMEOUT);
-        for (int i = 0; i < kSlotRing && i < cnt; ++i)   // let issued copies land
-          mbar_wait_bounded(&s_full[i], static_cast<uint32_t>((cnt - 1 - ((cnt - 1 - i) % kSlotRing)) / kSlotRing) & 1u);
+        for (int i = 0; i < kRing && i < cnt; ++i)   // let issued copies land
+          mbar_wait_bounded(&s_full[i], static_cast<uint32_t>((cnt - 1 - ((cnt - 1 - i) % kRing)) / kRing) & 1u);
       }
     }
   } else if (warp < 6) {
@@ -355,9 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = col0 >> lg_tw; t <= t_last; ++t) {   // 1 tile, or 2 when tile_w == 32
           if (t != cur_t) {                                // same for every thread of the CTA
             if constexpr (TSLOT) {
-              // tile t's record waits in ring slot scnt % kSlotRing (filled by TMA)
-              const int ring = scnt % kSlotRing;
-              if (!mbar_wait(&s_full[ring], static_cast<uint32_t>(scnt / kSlotRing) & 1u, abort_flag)) {
+              // tile t's record waits in ring slot scnt % kRing (filled by TMA)
+              const int ring = scnt % kRing;
+              if (!mbar_wait(&s_full[ring], static_cast<uint32_t>(scnt / kRing) & 1u, abort_flag)) {
                 ok = false;
                 break;
               }
@@ -376,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               // the previous slot's values are in registers by now: hand it back
               if (scnt > 0) {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[(scnt - 1) % kSlotRing]);
+                if (lane == 0) mbar_arrive(&s_empty[(scnt - 1) % kRing]);
               }
               ++scnt;
             } else {
@@ -666,13 +668,24 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   const int tile_m = pair ? 2 * kBlockM : kBlockM;
   P.num_m_blocks = (v.M + tile_m - 1) / tile_m;
   const size_t b_stage = pair ? kBBytes / 2 : kBBytes;
-  const size_t ring = tslot ? static_cast<size_t>(kSlotRing) * kBlockM * (2 * v.E + ib + 16) : 0;
-  const size_t fixed = 1024 + 512 + ring;
+  // Pipeline depth from the 227 KB budget.  A deep slot ring (4 hidden tiles)
+  // only pays while the A/B pipeline keeps at least 4 stages: at wide ell_w it
+  // is cut to 2, which leaves the MMA a free stage while the builders hold a
+  // whole hidden tile's K steps.
   const size_t budget = 227 * 1024;
-  int stages = static_cast<int>((budget - fixed) / (kABytes + b_stage));
-  if (stages > kMaxStages) stages = kMaxStages;
+  int ring_depth = kSlotRing, stages = 0;
+  size_t fixed = 0;
+  for (;;) {
+    const size_t ring = tslot ? static_cast<size_t>(ring_depth) * kBlockM * (2 * v.E + ib + 16) : 0;
+    fixed = 1024 + 512 + ring;
+    stages = static_cast<int>((budget - fixed) / (kABytes + b_stage));
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (!tslot || stages >= 4 || ring_depth == 2) break;
+    --ring_depth;
+  }
   if (stages < 2) return cudaErrorInvalidValue;
   P.stages = stages;
+  P.ring = ring_depth;
   const size_t smem = fixed + static_cast<size_t>(stages) * (kABytes + b_stage);
   switch (ev) {
     case 1: return launch_down_ev<1>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);

@@ -139,7 +139,8 @@ twell_status up_pack_checked(const uint16_t *x, const uint16_t *W_up, const uint
   UpArgs a;
   a.x = x; a.w_up = W_up; a.w_gate = W_gate; a.b = b;
   a.M = M; a.d = d_model; a.f = d_ff; a.z_debug = z_debug;
-  cudaError_t e = launch_up_pack(a, t, sms, s);
+  cudaError_t e = decode_up_eligible(M, d_ff, tile_w) ? launch_up_pack_decode(a, t, sms, s)
+                                                       : launch_up_pack(a, t, sms, s);
   if (e != cudaSuccess) return TWELL_ERR_CUDA;
   return from_cuda(launch_overflow_finalize(t, s));
 }
@@ -186,6 +187,8 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
   const int sms = sm_count();
   if (sms <= 0) return TWELL_ERR_CUDA;
   if (mode == TWELL_DOWN_GATHER) return from_cuda(launch_spmm_gather(v, W_down, d_model, y, nullptr, s));
+  // decode-size batches: the split-K tensor-core kernel streams W_down over every SM
+  if (decode_down_eligible(a->M)) return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, s));
   if (mode == TWELL_DOWN_MMA) return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, s));
   const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);

@@ -93,6 +93,14 @@ cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
                             const int32_t *blk_path, int num_sms, cudaStream_t s);
 
+// Decode-size batches (M <= 256): tokens on the MMA N side, weights streamed
+// over all SMs (up: one CTA per 128 hidden units; down: split-K clusters).
+bool decode_up_eligible(int M, int d_ff, int tile_w);
+bool decode_down_eligible(int M);
+cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
+cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
+                               int num_sms, cudaStream_t s);
+
 // Density (nonzeros / (rows * d_ff)) of a 128-token block at or above which the
 // AUTO down-projection uses the tensor-core path.  Chosen from measurement.
 constexpr float kDownCrossoverDensity = 0.006f;

@@ -1,0 +1,126 @@
+"""GPU parity of the decode-size kernels (M <= 256 tokens: tokens on the MMA's N
+side, split-K clusters for the down-projection) against the CPU oracle.
+
+Batches of at most 256 tokens are routed to these kernels by the library
+(twell_up_pack when tile_w <= 128 and d_ff % 128 == 0; twell_spmm in the
+tensor-core and automatic modes), so every case below runs them.  Cases cover
+single-token and ragged batches, every tile width, the gated form, ell_w that is
+not a multiple of 8 or above 32, heavy overflow, d_model that ends half-way into
+a 128-column slice, and d_ff that ends inside a 64-column K step.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import twell_synth as S
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import activation_sparse_ffn_twell_b200 as T
+    from _gpu_helpers import (assert_twell_equal, assert_y_close, dev, h_from_zdebug, host_bits,
+                              twell_to_np, upload_twell)
+
+GEMM_REL_BOUND = 2.0 ** -16
+
+UP_CASES = [
+    # M, d, f, tw, E, rho, gated
+    (1, 256, 1024, 128, 16, 0.05, False),
+    (5, 192, 512, 64, 8, 0.10, False),
+    (16, 128, 256, 32, 8, 0.10, False),
+    (33, 256, 1024, 128, 12, 0.20, False),     # E not a multiple of 8, overflow
+    (100, 128, 512, 128, 40, 0.30, False),     # E > 32: two padding passes
+    (256, 256, 2048, 128, 8, 0.15, False),     # largest decode batch, heavy overflow
+    (7, 128, 512, 128, 16, 0.05, True),
+    (64, 256, 512, 64, 8, 0.10, True),
+    (250, 128, 256, 32, 8, 0.15, True),
+    (40, 64, 256, 64, 64, 0.50, False),        # E == tile_w: no overflow possible
+    (48, 128, 384, 64, 8, 1.0, False),         # every pair overflows
+]
+
+
+@pytest.mark.parametrize("M,d,f,tw,E,rho,gated", UP_CASES)
+def test_decode_up_pack_bitexact_given_accumulators(M, d, f, tw, E, rho, gated):
+    L = S.small_random(M, d, f, tw, E, rho, gated=gated, seed=M * 31 + d + f)
+    z = torch.zeros((M, 2 * f if gated else f), dtype=torch.float32, device="cuda")
+    a = T.twell_up_pack(dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_gate), tile_w=tw, ell_w=E,
+                        ovf_capacity=M * (f // tw), z_debug=z)
+    code, n = T.read_status(a)
+    assert code == 0
+    zg = z.cpu().numpy()
+    h_gpu = h_from_zdebug(zg, L.b, gated, f)
+    ref = O.twell_pack(h_gpu, tw, E)
+    got, _ = twell_to_np(a)
+    assert n == ref.n_ovf
+    assert_twell_equal(got, ref)
+    x = O.bits_to_f64(L.x)
+    for name, w in (("gate", L.w_gate), ("up", L.w_up)) if gated else (("up", L.w_up),):
+        W = O.bits_to_f64(w)
+        bound = GEMM_REL_BOUND * (np.abs(x) @ np.abs(W).T) + 1e-30
+        zz = zg[:, :f] if (not gated or name == "gate") else zg[:, f:]
+        assert (np.abs(zz - x @ W.T) / bound).max() <= 1.0, name
+
+
+DOWN_CASES = [
+    # M, d, f, tw, E, rho
+    (1, 256, 1024, 128, 16, 0.05),
+    (17, 64, 512, 64, 8, 0.10),        # d_model = 64: half of one 128-column slice
+    (64, 192, 1024, 128, 16, 0.10),    # second slice half outside d_model
+    (200, 1024, 2048, 256, 24, 0.05),
+    (256, 512, 1024, 128, 8, 0.30),    # heavy overflow
+    (90, 256, 96, 32, 4, 0.10),        # d_ff = 96 ends inside a K step
+    (120, 256, 512, 128, 5, 0.05),     # E not a multiple of 8
+    (48, 128, 512, 64, 8, 1.0),        # every pair overflows
+    (32, 4096, 2048, 128, 8, 0.02),    # 32 slices: split-K over 4-CTA clusters
+]
+
+
+@pytest.mark.parametrize("mode", ["mma", "auto"])
+@pytest.mark.parametrize("M,d,f,tw,E,rho", DOWN_CASES)
+def test_decode_spmm(M, d, f, tw, E, rho, mode):
+    L = S.small_random(M, d, f, tw, E, rho, seed=M * 5 + d + 3 * f)
+    h = O.hidden(L.x, L.w_up, L.b, L.w_gate)
+    ref = O.twell_pack(h, tw, E)
+    a = upload_twell(ref, cap=max(ref.n_ovf, 1))
+    y = T.twell_spmm(a, dev(L.w_down), mode=mode)
+    assert T.read_status(a)[0] == 0
+    assert_y_close(y, O.twell_spmm(ref, L.w_down))
+
+
+def test_decode_spmm_zero_density_is_exact_zero():
+    L = S.small_random(100, 512, 1024, 128, 16, 0.0)
+    ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), 128, 16)
+    a = upload_twell(ref, cap=1)
+    y = T.twell_spmm(a, dev(L.w_down), mode="mma")
+    assert torch.count_nonzero(y.float()).item() == 0
+
+
+@pytest.mark.parametrize("M", [1, 77, 256])
+@pytest.mark.parametrize("gated", [False, True])
+def test_decode_integer_family_forward_bitexact(M, gated):
+    """Integer-valued layers: fp32 sums are exact in any order, so the fused
+    decode forward (split-K partials included) must equal the oracle bitwise."""
+    L = S.integer_exact(M=M, d_model=512, d_ff=2048, tile_w=128, density=0.05, gated=gated,
+                        seed=M)
+    ref, y64 = O.ffn_forward(L.x, L.w_up, L.b, L.w_down, L.tile_w, L.ell_w, L.w_gate)
+    y, a = T.twell_ffn_forward(dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_down), tile_w=L.tile_w,
+                               ell_w=L.ell_w, W_gate=dev(L.w_gate), mode="auto",
+                               ovf_capacity=max(ref.n_ovf, 1))
+    assert T.read_status(a) == (0, ref.n_ovf)
+    got, _ = twell_to_np(a)
+    assert_twell_equal(got, ref)
+    assert np.array_equal(host_bits(y), O.f64_to_bits(O.bf16_round(y64)))
+
+
+def test_decode_and_gather_agree_on_the_same_twell():
+    """The split-K kernel and the CUDA-core gather read the same TwELL; both are
+    within tolerance of the oracle, and of each other."""
+    L = S.small_random(128, 1024, 4096, 128, 16, 0.02, seed=11)
+    ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), 128, 16)
+    a = upload_twell(ref, cap=max(ref.n_ovf, 1))
+    y_ref = O.twell_spmm(ref, L.w_down)
+    y_mma = T.twell_spmm(a, dev(L.w_down), mode="mma")
+    y_gat = T.twell_spmm(a, dev(L.w_down), mode="gather")
+    assert_y_close(y_mma, y_ref)
+    assert_y_close(y_gat, y_ref)

@@ -114,6 +114,11 @@ SPMM_CASES = [
     (130, 2048, 1024, 256, 24, 0.05),
     (200, 256, 512, 128, 5, 0.05),     # ell_w not a multiple of 8
     (96, 128, 512, 64, 8, 1.0),        # every pair overflows
+    # more than 256 tokens: the token-major tensor-core kernel (fewer go to the
+    # split-K decode kernel)
+    (300, 256, 512, 128, 5, 0.05),     # ell_w not a multiple of 8
+    (290, 128, 512, 64, 8, 1.0),       # every pair overflows
+    (260, 1024, 1024, 32, 8, 0.10),
 ]
 
 
@@ -151,6 +156,11 @@ UP_CASES = [
     (200, 256, 1024, 128, 16, 0.05, True),
     (150, 128, 512, 64, 8, 0.10, True),
     (70, 128, 256, 32, 8, 0.15, True),
+    # more than 256 tokens: the token-major producer (fewer go to the decode kernel)
+    (300, 256, 1024, 128, 16, 0.05, False),
+    (333, 128, 512, 32, 8, 0.10, False),
+    (390, 128, 512, 64, 8, 0.10, True),
+    (280, 128, 512, 128, 12, 0.20, True),
 ]
 
 
