@@ -54,9 +54,6 @@ struct DecUpParams {
   int np;                 // MMA N: tokens rounded up to a multiple of 16
   int acc_up;             // TMEM column of the up-branch accumulator (gated)
   int num_kb, num_ub, stages;
-  int ksub;               // 64-wide K steps per pipeline stage (1, 2 or 4)
-  int pf;                 // K steps of weights prefetched into L2 ahead of the ring
-  int stagger;            // 1: CTA ub starts its K loop at an offset proportional to ub
   uint32_t tmem_cols, idesc;
   float *z_debug;
   PackTarget out;
@@ -72,11 +69,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int kStages = P.stages;
-  // a stage holds ksub consecutive K steps, each [W_up tile][W_gate tile][x tile]:
-  // the weight rows are then read ksub x 128 bytes at a time
-  const int SUB = W_BYTES + P.np * 128;
-  const int STAGE = P.ksub * SUB;
-  const int n_groups = (P.num_kb + P.ksub - 1) / P.ksub;
+  const int STAGE = W_BYTES + P.np * 128;                 // [W_up tile][W_gate tile][x tile]
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * STAGE);
   uint64_t *full = bars;
   uint64_t *empty = bars + kDecMaxStages;
@@ -116,38 +109,16 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
       uint32_t filled = 0;
       bool ok = true;
       for (int ub = blockIdx.x; ub < P.num_ub && ok; ub += gridDim.x) {
-        // weight rows of the next P.pf K steps go to L2 ahead of the ring, so
-        // that more of this SM's share of the weights is in flight
-        for (int kb = 0; kb < P.pf && kb < P.num_kb; ++kb) {
-          tma_prefetch_l2_2d(&tmap_w, kb * kBlockK, ub * kDecUnits);
-          if constexpr (GATED) tma_prefetch_l2_2d(&tmap_g, kb * kBlockK, ub * kDecUnits);
-        }
-        const int kg_start = P.stagger ? static_cast<int>((static_cast<long long>(ub) * n_groups) / P.num_ub) : 0;
-        for (int i = 0; i < n_groups; ++i) {
+        for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          int kg = kg_start + i;
-          if (kg >= n_groups) kg -= n_groups;
-          const int kb0 = kg * P.ksub;
-          for (int j = 0; j < P.ksub; ++j) {
-            const int kp = kb0 + j + P.pf;
-            if (P.pf > 0 && kp < P.num_kb) {
-              tma_prefetch_l2_2d(&tmap_w, kp * kBlockK, ub * kDecUnits);
-              if constexpr (GATED) tma_prefetch_l2_2d(&tmap_g, kp * kBlockK, ub * kDecUnits);
-            }
-          }
-          const int nsub = min(P.ksub, P.num_kb - kb0);
           // the x box is M rows; operand rows M..np-1 feed accumulator columns
           // that no one reads
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nsub * (W_BYTES + P.M * 128)));
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(W_BYTES + P.M * 128));
           filled |= 1u << stage;
-          for (int j = 0; j < nsub; ++j) {   // weight boxes first: one burst per row
-            uint8_t *dst = smem + stage * STAGE + j * SUB;
-            tma_load_2d(dst, &tmap_w, &full[stage], (kb0 + j) * kBlockK, ub * kDecUnits);
-            if constexpr (GATED)
-              tma_load_2d(dst + kWBytes, &tmap_g, &full[stage], (kb0 + j) * kBlockK, ub * kDecUnits);
-          }
-          for (int j = 0; j < nsub; ++j)
-            tma_load_2d(smem + stage * STAGE + j * SUB + W_BYTES, &tmap_x, &full[stage], (kb0 + j) * kBlockK, 0);
+          uint8_t *dst = smem + stage * STAGE;
+          tma_load_2d(dst, &tmap_w, &full[stage], kb * kBlockK, ub * kDecUnits);
+          if constexpr (GATED) tma_load_2d(dst + kWBytes, &tmap_g, &full[stage], kb * kBlockK, ub * kDecUnits);
+          tma_load_2d(dst + W_BYTES, &tmap_x, &full[stage], kb * kBlockK, 0);
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -169,26 +140,20 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
       for (int ub = blockIdx.x; ub < P.num_ub && ok; ub += gridDim.x, ++it) {
         if (!mbar_wait(tm_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const int kg_start = P.stagger ? static_cast<int>((static_cast<long long>(ub) * n_groups) / P.num_ub) : 0;
-        for (int i = 0; i < n_groups; ++i) {
+        for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          int kg = kg_start + i;
-          if (kg >= n_groups) kg -= n_groups;
-          const int nsub = min(P.ksub, P.num_kb - kg * P.ksub);
-          for (int j = 0; j < nsub; ++j) {
-            const uint32_t w_addr = smem_u32(smem + stage * STAGE + j * SUB);
-            const uint32_t x_addr = w_addr + W_BYTES;
+          const uint32_t w_addr = smem_u32(smem + stage * STAGE);
+          const uint32_t x_addr = w_addr + W_BYTES;
 #pragma unroll
-            for (int k = 0; k < kBlockK / kUmmaK; ++k) {
-              const uint64_t xdesc = smem_desc_sw128(x_addr + k * 32, 16, 1024);
-              const uint32_t acc = (i | j | k) != 0;
-              if constexpr (GATED) {
-                umma_bf16(tmem_base, smem_desc_sw128(w_addr + kWBytes + k * 32, 16, 1024), xdesc, P.idesc, acc);
-                umma_bf16(tmem_base + P.acc_up, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
-              } else {
-                umma_bf16(tmem_base, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
-              }
+          for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+            const uint64_t xdesc = smem_desc_sw128(x_addr + k * 32, 16, 1024);
+            const uint32_t acc = (kb | k) != 0;
+            if constexpr (GATED) {
+              umma_bf16(tmem_base, smem_desc_sw128(w_addr + kWBytes + k * 32, 16, 1024), xdesc, P.idesc, acc);
+              umma_bf16(tmem_base + P.acc_up, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
+            } else {
+              umma_bf16(tmem_base, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
             }
           }
           umma_commit(&empty[stage]);
@@ -348,7 +313,6 @@ struct DecDownParams {
   int num_kb;             // hidden K steps of 64
   int split;              // CTAs per cluster (K ranges per 128 output columns)
   int stages;
-  int pf;                 // K steps of W_down prefetched into L2 ahead of the ring
   uint32_t tmem_cols, idesc;
 };
 
@@ -407,16 +371,8 @@ __global__ void __launch_bounds__(kDecDownThreads, 1)
       int stage = 0; uint32_t phase = 0;
       uint32_t filled = 0;
       bool ok = true;
-      for (int kb = kb_lo; kb < kb_hi && kb < kb_lo + P.pf; ++kb) {   // W_down rows to L2 ahead
-        tma_prefetch_l2_2d(&tmap_wd, col0, kb * kBlockK);
-        tma_prefetch_l2_2d(&tmap_wd, col0 + 64, kb * kBlockK);
-      }
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-        if (P.pf > 0 && kb + P.pf < kb_hi) {
-          tma_prefetch_l2_2d(&tmap_wd, col0, (kb + P.pf) * kBlockK);
-          tma_prefetch_l2_2d(&tmap_wd, col0 + 64, (kb + P.pf) * kBlockK);
-        }
         mbar_arrive_expect_tx(&full[stage], kWBytes);
         filled |= 1u << stage;
         uint8_t *dst = smem + stage * STAGE;
@@ -657,40 +613,8 @@ __global__ void __launch_bounds__(kDecDownThreads, 1)
 
 int round_tokens(int M) { return M <= 16 ? 16 : (M + 15) & ~15; }
 
-// Largest number of 64-wide K steps the decode up-projection groups into one
-// pipeline stage (TWELL_DEC_KSUB = 1, 2 or 4; a tuning knob, default 4).
-int dec_ksub_limit() {
-  static int v = 0;
-  if (v == 0) {
-    const char *e = getenv("TWELL_DEC_KSUB");
-    const int r = (e != nullptr) ? atoi(e) : 4;
-    v = (r == 1 || r == 2 || r == 4) ? r : 4;
-  }
-  return v;
-}
 
-// K steps of weights the decode kernels prefetch into L2 ahead of their
-// shared-memory ring (TWELL_DEC_PF; a tuning knob).
-int dec_prefetch() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("TWELL_DEC_PF");
-    const int r = (e != nullptr) ? atoi(e) : 0;
-    v = (r >= 0 && r <= 64) ? r : 0;
-  }
-  return v;
-}
 
-// 1: the decode up-projection rotates each CTA's K order (TWELL_DEC_STAGGER;
-// a tuning knob).
-int dec_stagger() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("TWELL_DEC_STAGGER");
-    v = (e != nullptr && e[0] == '1') ? 1 : 0;
-  }
-  return v;
-}
 
 template <int TW, bool GATED>
 cudaError_t launch_up_dec_impl(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s) {
@@ -706,15 +630,8 @@ cudaError_t launch_up_dec_impl(const UpArgs &a, const PackTarget &t, int num_sms
   P.num_ub = a.f / kDecUnits;
   P.z_debug = a.z_debug;
   P.out = t;
-  const size_t sub = (GATED ? 2 : 1) * static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
+  const size_t stage = (GATED ? 2 : 1) * static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
   const size_t extra = 1024 + 4096;                      // alignment slack, barriers, counts
-  // K steps per stage: grouped while the pipeline still gets 2 stages
-  int ksub = dec_ksub_limit();
-  while (ksub > 1 && (kDecSmemBudget - extra) / (ksub * sub) < 2) ksub >>= 1;
-  P.ksub = ksub;
-  P.pf = dec_prefetch();
-  P.stagger = dec_stagger();
-  const size_t stage = ksub * sub;
   int stages = static_cast<int>((kDecSmemBudget - extra) / stage);
   if (stages > kDecMaxStages) stages = kDecMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
@@ -849,7 +766,6 @@ cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d
     if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = split; }
   }
   P.split = best;
-  P.pf = dec_prefetch();
   CUtensorMap mw;
   if (encode_tensor_map_2d(&mw, w_down, d, v.f, static_cast<uint64_t>(d) * 2, 64, kBlockK,
                            CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)

@@ -8,20 +8,27 @@
 // the dense backup segment of overflowing pairs) -- the dense h never exists in
 // HBM -- and multiplied by the matching 64 rows of W_down.
 //
-// Roles (one CTA per SM, persistent over 128-token x 256-column tiles of y):
+// Roles (one CTA per SM, persistent over 128-token x 256- or 512-column tiles
+// of y):
 //   warp 0      TMA: W_down[k0:k0+64, n0:n0+256] as four 64x64 boxes, 128-byte
-//               swizzle; this is an N-major ("MN-major") B operand.
-//   warp 1      TMEM allocation (2 x 256 fp32 columns) + tcgen05.mma issue.
+//               swizzle; this is an N-major ("MN-major") B operand.  512-column
+//               tiles load two such stages per K step from their own ring.
+//   warp 1      TMEM allocation (512 fp32 columns: two 256-column accumulators,
+//               double-buffered, or both halves of one 512-column tile) +
+//               tcgen05.mma issue.
 //   warps 2..5  epilogue: TMEM -> fp32 registers -> bf16 -> y.
-//   warps 6..9  A builders: thread = token row.  Fast path (ell_w % 8 == 0):
-//               the row's slot record of the next hidden tile is loaded into
-//               registers with 128/64-bit loads while the current one is used;
-//               the K steps of one tile are claimed together (the TMA warp
-//               has already cleared them with a bulk copy of zeros), and each
-//               slot is written once with a predicated 2-byte store (fully
-//               unrolled over ell_w).
-//               General path: per K step, zero the row and scatter from global
-//               memory.  Then fence to the async proxy and arrive.
+//   warps 6..13 A builders.  Fast path (ell_w % 8 == 0): two threads per token
+//               row, each taking alternate slots.  The row's slot record of the
+//               next hidden tile is in registers (or a TMA-fed shared-memory
+//               ring, warp 14) before it is needed; the K steps of one tile are
+//               claimed together as soon as the MMA releases them, each thread
+//               clears its half of the row, and each slot is written once with
+//               a predicated 2-byte store (fully unrolled over ell_w).
+//               General path (warps 6..9, thread = row): per K step, zero the
+//               row and scatter from global memory.  Then fence to the async
+//               proxy and arrive.
+//   warp 14     slot producer: TMA boxes of the 128 rows' slot records per
+//               hidden tile into the ring.
 #include <cstdlib>
 
 #include "twell_device.cuh"
@@ -39,17 +46,14 @@ constexpr int kThreads = 480;
 constexpr int kSlotWarp = 14;
 constexpr int kSlotRing = 4;                    // max slot-record ring depth (hidden tiles)
 
-// Source of the per-stage A clear: the fast builders only write nonzeros, the
-// TMA engine zeroes the stage first (a bulk copy from this never-written array),
-// which keeps 16 KB per K step off the threads' shared-memory store path.
-__device__ __align__(128) uint8_t g_zero_tile[kBlockM * kBlockK * 2];
 
 struct DownParams {
   TwellView A;
   uint16_t *y;
   int d;
   int num_m_blocks, num_n_blocks, num_kb;
-  int stages;                // pipeline depth (<= kMaxStages), set from shared-memory budget
+  int stages;                // A pipeline depth (<= kMaxStages), set from shared-memory budget
+  int bstages;               // W_down pipeline depth (== stages unless WIDE)
   int slot_ib;               // bytes of the index box per row (covers ell_w indices)
   int ring;                  // slot-record ring depth (2..kSlotRing)
   const int32_t *blk_path;   // NULL, or per 128-token block: 1 = this path owns it
@@ -75,11 +79,18 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
 // PAIR: a cluster of 2 CTAs computes a 256-token x 256-column tile with M=256
 // MMAs (cta_group::2); each CTA builds its 128 rows of A and loads half of the
 // W_down columns, so each SM carries half the B operand traffic.
-template <int EV, bool TSLOT, bool PAIR>
+// WIDE (single CTA only): a tile is 128 tokens x 512 y columns -- both halves
+// of TMEM -- so each rebuilt A stage feeds two 256-column MMAs, from a separate
+// ring of W_down stages.  Half as many A rebuilds per FLOP, and twice the MMA
+// time to hide each one behind.
+template <int EV, bool TSLOT, bool PAIR, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_spmm_mma(const __grid_constant__ CUtensorMap tmap_wd, const __grid_constant__ CUtensorMap tmap_sv,
                const __grid_constant__ CUtensorMap tmap_si, const __grid_constant__ CUtensorMap tmap_sn,
                const DownParams P) {
+  static_assert(!(WIDE && PAIR), "512-column tiles are single-CTA");
+  constexpr int NH = WIDE ? 2 : 1;                            // 256-column halves per tile
+  constexpr int kTN = NH * kBN;                               // y columns per tile
   constexpr int TILE_M = PAIR ? 2 * kBlockM : kBlockM;
   constexpr int B_BYTES = PAIR ? kBBytes / 2 : kBBytes;      // this CTA's W_down columns
   constexpr int B_BOXES = PAIR ? kBN / 128 : kBN / 64;        // 64-column TMA boxes per CTA
@@ -88,9 +99,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int kStages = P.stages;
+  const int kBStages = P.bstages;
   uint8_t *sA = smem;
   uint8_t *sB = smem + kStages * kABytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kStages * B_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kBStages * B_BYTES);
   uint64_t *full = bars;
   uint64_t *empty = bars + kMaxStages;
   uint64_t *tm_full = bars + 2 * kMaxStages;
@@ -98,8 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *drain = bars + 2 * kMaxStages + 4;
   uint64_t *s_full = bars + 2 * kMaxStages + 5;               // slot ring
   uint64_t *s_empty = s_full + kSlotRing;
-  uint64_t *zfull = s_empty + kSlotRing;                        // A stage cleared by TMA
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(zfull + kMaxStages);
+  uint64_t *bfull = s_empty + kSlotRing;                        // W_down ring (WIDE)
+  uint64_t *bempty = bfull + kMaxStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bempty + kMaxStages);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   // slot ring entry: [128][ell_w] bf16 values, [128][slot_ib] u8 indices, [128][8] u16 nnz
   uint8_t *sRing = reinterpret_cast<uint8_t *>(bars) + 512;
@@ -119,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) { mbar_init(&tm_full[i], 1); mbar_init(&tm_empty[i], PAIR ? 8 : 4); }
     for (int i = 0; i < kSlotRing; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 8); }
-    for (int i = 0; i < kStages; ++i) mbar_init(&zfull[i], 1);
+    if (WIDE) for (int i = 0; i < kBStages; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -145,18 +158,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ TMA (W_down)
     if (lane == 0) {
       int stage = 0; uint32_t phase = 0; uint32_t filled = 0;
+      int bst = 0; uint32_t bph = 0; uint32_t bfilled = 0;   // W_down ring (WIDE)
       bool ok = true;
       for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
         const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
+        if constexpr (WIDE) {
+          for (int kb = 0; kb < P.num_kb && ok; ++kb) {
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+            filled |= 1u << stage;
+            mbar_arrive(&full[stage]);   // (no bytes: the builders fill A)
+            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+            for (int h = 0; h < NH; ++h) {
+              if (!mbar_wait(&bempty[bst], bph ^ 1u, abort_flag)) { ok = false; break; }
+              mbar_arrive_expect_tx(&bfull[bst], B_BYTES);
+              bfilled |= 1u << bst;
+              uint8_t *dst = sB + bst * B_BYTES;
+#pragma unroll
+              for (int j = 0; j < B_BOXES; ++j)
+                tma_load_2d(dst + j * (kBlockK * 128), &tmap_wd, &bfull[bst], n_blk * kTN + h * kBN + j * 64,
+                            kb * kBlockK);
+              if (++bst == kBStages) { bst = 0; bph ^= 1u; }
+            }
+          }
+          continue;
+        }
         for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * B_BYTES);
           filled |= 1u << stage;
-          if constexpr (EV > 0) {   // clear this CTA's A stage for its builders
-            mbar_arrive_expect_tx(&zfull[stage], kABytes);
-            bulk_load(sA + stage * kABytes, g_zero_tile, kABytes, &zfull[stage]);
-          }
           uint8_t *dst = sB + stage * B_BYTES;
           const int col_b = n_blk * kBN + static_cast<int>(rank) * (B_BOXES * 64);
 #pragma unroll
@@ -176,8 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         raise_status(A.status, TWELL_ERR_TIMEOUT);
         for (int i = 0; i < kStages; ++i) {
           if (!((filled >> i) & 1u)) continue;
-          if (leader) mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
-          if (EV > 0) mbar_wait_bounded(&zfull[i], (i < stage) ? phase : (phase ^ 1u));
+          if (leader && !WIDE) mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
+        }
+        for (int i = 0; WIDE && i < kBStages; ++i) {
+          if (!((bfilled >> i) & 1u)) continue;
+          mbar_wait_bounded(&bfull[i], (i < bst) ? bph : (bph ^ 1u));
         }
       }
     }
@@ -185,16 +218,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
       int stage = 0; uint32_t phase = 0; int it = 0;
+      int bst = 0; uint32_t bph = 0;   // W_down ring (WIDE)
       bool ok = true;
       for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
         const int m_blk = tile % P.num_m_blocks;
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        // WIDE: one accumulator set (both TMEM halves); else two, alternating
+        const int acc = WIDE ? 0 : (it & 1);
+        const uint32_t acc_phase = WIDE ? (it & 1) : ((it >> 1) & 1);
         ++it;
         if (!mbar_wait<PAIR>(&tm_empty[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        if constexpr (WIDE) {
+          for (int kb = 0; kb < P.num_kb && ok; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + stage * kABytes);
+            for (int h = 0; h < NH; ++h) {
+              if (!mbar_wait(&bfull[bst], bph, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t b_addr = smem_u32(sB + bst * B_BYTES);
+#pragma unroll
+              for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+                const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
+                const uint64_t bdesc = smem_desc_sw128(b_addr + k * 2048, kBlockK * 128, 1024);
+                umma_bf16(d_tmem + h * kBN, adesc, bdesc, IDESC, (kb | k) != 0);
+              }
+              umma_commit(&bempty[bst]);
+              if (++bst == kBStages) { bst = 0; bph ^= 1u; }
+            }
+            umma_commit(&empty[stage]);   // the A stage may be rebuilt
+            if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          umma_commit(&tm_full[acc]);
+          continue;
+        }
         for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -261,8 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = unit0; tile < num_tiles; tile += n_units) {
       const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
       if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = WIDE ? 0 : (it & 1);
+      const uint32_t acc_phase = WIDE ? (it & 1) : ((it >> 1) & 1);
       ++it;
       if (!mbar_wait<PAIR>(&tm_full[acc], acc_phase, abort_flag)) {
         *abort_flag = 1;
@@ -273,14 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = m_blk * TILE_M + row_base + row_in_tile;
       const bool valid = r < A.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
-      uint16_t *yr = P.y + static_cast<size_t>(r) * P.d + n_blk * kBN;
+      uint16_t *yr = P.y + static_cast<size_t>(r) * P.d + n_blk * kTN;
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < kTN / 32; ++c) {
         uint32_t v[32];
         __syncwarp();
         tmem_ld_32x32b_x32(t_row + c * 32, v);
         tmem_ld_wait();
-        if (valid && n_blk * kBN + c * 32 < P.d) {
+        if (valid && n_blk * kTN + c * 32 < P.d) {
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             uint4 o;
@@ -302,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if constexpr (EV > 0) {
     // ------------------------------------------------------------ A builders (fast)
     // ell_w == 8*EV.  Per hidden tile, the row's slot record (values, indices,
-    // nnz) is loaded into registers one tile ahead; the tile's K steps are zeroed
+    // nnz) is in registers before it is needed; the tile's K steps are cleared
     // with independent 16-byte stores and every slot is written once with a
     // predicated 2-byte store -- a fully unrolled, dependency-free sequence.
     constexpr int E = 8 * EV;
@@ -316,7 +376,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     int stage = 0; uint32_t phase = 0;
     int scnt = 0;   // slot-ring records consumed so far (TSLOT)
     bool ok = true;
-    for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
+    // The eight builder warps meet at a named barrier once per group of K
+    // steps; a bounded wait that gives up is OR-ed into that barrier so they all
+    // leave at the same group (no warp is left waiting for the others).
+    for (int tile = unit0; tile < num_tiles; tile += n_units) {
       const int m_blk = tile % P.num_m_blocks;
       if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
       const int r = m_blk * TILE_M + row_base + row_in_tile;
@@ -344,14 +407,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the ring holds them) so every slot is visited once per tile
       // (at most stages-1 of them, so the MMA always has a stage to work on)
       const int S = max(1, min(tw / kBlockK, kStages - 1));
-      for (int kb0 = 0; kb0 < P.num_kb && ok; kb0 += S) {
+      for (int kb0 = 0; kb0 < P.num_kb; kb0 += S) {
         const int nsteps = min(S, P.num_kb - kb0);
         const int stage0 = stage;
-        for (int j = 0; j < nsteps; ++j) {   // each step's A buffer, already zeroed by TMA
-          if (!mbar_wait(&zfull[stage], phase, abort_flag)) { ok = false; break; }
+        // claim the group's A stages as soon as the MMA has released them and
+        // clear this thread's half of its row (row-XOR chunk order: the 32 rows
+        // of a warp hit all banks)
+        bool fail = !ok;
+        for (int j = 0; j < nsteps; ++j) {
+          if (!fail && !mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) fail = true;
+          if (!fail) {
+            uint8_t *rowA = sA + stage * kABytes + row_in_tile * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4 *>(rowA + (((4 * half + c) ^ static_cast<int>(row_swz)) << 4)) =
+                  make_uint4(0u, 0u, 0u, 0u);
+          }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
+        fence_proxy_async_smem();   // the zeros precede any backup copy by the async proxy
+        if (named_bar_any(1, 256, fail)) { ok = false; break; }
         const int col0 = kb0 * kBlockK, span = nsteps * kBlockK;
         const int t_last = (col0 + span - 1) >> lg_tw;
         for (int t = col0 >> lg_tw; t <= t_last; ++t) {   // 1 tile, or 2 when tile_w == 32
@@ -457,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      if (!ok) break;   // every builder warp left at the same barrier
     }
     if (!ok) {
       *abort_flag = 1;
@@ -560,11 +636,11 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
   }
 }
 
-template <int EV, bool TSLOT, bool PAIR>
+template <int EV, bool TSLOT, bool PAIR, bool WIDE = false>
 cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUtensorMap &si,
                         const CUtensorMap &sn, const DownParams &P, int num_sms, size_t smem,
                         cudaStream_t s) {
-  auto kern = k_spmm_mma<EV, TSLOT, PAIR>;
+  auto kern = k_spmm_mma<EV, TSLOT, PAIR, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -597,9 +673,15 @@ cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUte
 }
 
 template <int EV>
-cudaError_t launch_down_ev(bool tslot, bool pair, const CUtensorMap &mw, const CUtensorMap &sv,
+cudaError_t launch_down_ev(bool tslot, bool pair, bool wide, const CUtensorMap &mw, const CUtensorMap &sv,
                            const CUtensorMap &si, const CUtensorMap &sn, const DownParams &P,
                            int num_sms, size_t smem, cudaStream_t s) {
+  if (wide) {
+    if constexpr (EV > 0) {
+      if (tslot) return launch_down<EV, true, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+    }
+    return launch_down<EV, false, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+  }
   if constexpr (EV > 0) {
     if (pair) {
       return tslot ? launch_down<EV, true, true>(mw, sv, si, sn, P, num_sms, smem, s)
@@ -623,6 +705,16 @@ bool down_uses_pair(const TwellView &v) {
     env = (e != nullptr && e[0] == '1') ? 1 : 0;
   }
   return env == 1 && v.E % 8 == 0 && v.E <= 64;
+}
+
+// 512-column tiles are on unless TWELL_DOWN_WIDE=0 (a tuning / comparison knob).
+bool down_uses_wide() {
+  static int env = -1;
+  if (env < 0) {
+    const char *e = getenv("TWELL_DOWN_WIDE");
+    env = (e != nullptr && e[0] == '0') ? 0 : 1;
+  }
+  return env == 1;
 }
 
 cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s) {
@@ -665,38 +757,52 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   }
   P.slot_ib = ib;
   const bool pair = down_uses_pair(v);
+  // 512-column tiles unless y has at most 256 columns (or CTA pairs are on):
+  // measured 1.7x the throughput of 256-column tiles per y column, which
+  // outweighs a worse-filled last wave of SMs
+  const bool wide = !pair && d > kBN && down_uses_wide();
   const int tile_m = pair ? 2 * kBlockM : kBlockM;
   P.num_m_blocks = (v.M + tile_m - 1) / tile_m;
+  P.num_n_blocks = (d + (wide ? 2 : 1) * kBN - 1) / ((wide ? 2 : 1) * kBN);
   const size_t b_stage = pair ? kBBytes / 2 : kBBytes;
   // Pipeline depth from the 227 KB budget.  A deep slot ring (4 hidden tiles)
-  // only pays while the A/B pipeline keeps at least 4 stages: at wide ell_w it
-  // is cut to 2, which leaves the MMA a free stage while the builders hold a
-  // whole hidden tile's K steps.
+  // only pays while the pipeline keeps at least 4 stages: at wide ell_w it is
+  // cut to 2, which leaves the MMA a free stage while the builders hold a
+  // whole hidden tile's K steps.  WIDE: 4 A stages, the rest W_down stages.
   const size_t budget = 227 * 1024;
-  int ring_depth = kSlotRing, stages = 0;
+  int ring_depth = kSlotRing, stages = 0, bstages = 0;
   size_t fixed = 0;
   for (;;) {
     const size_t ring = tslot ? static_cast<size_t>(ring_depth) * kBlockM * (2 * v.E + ib + 16) : 0;
     fixed = 1024 + 512 + ring;
-    stages = static_cast<int>((budget - fixed) / (kABytes + b_stage));
-    if (stages > kMaxStages) stages = kMaxStages;
-    if (!tslot || stages >= 4 || ring_depth == 2) break;
+    if (wide) {
+      stages = 4;
+      bstages = static_cast<int>((budget - fixed - stages * static_cast<size_t>(kABytes)) / b_stage);
+      if (bstages > kMaxStages) bstages = kMaxStages;
+      if (!tslot || bstages >= 4 || ring_depth == 2) break;
+    } else {
+      stages = static_cast<int>((budget - fixed) / (kABytes + b_stage));
+      if (stages > kMaxStages) stages = kMaxStages;
+      bstages = stages;
+      if (!tslot || stages >= 4 || ring_depth == 2) break;
+    }
     --ring_depth;
   }
-  if (stages < 2) return cudaErrorInvalidValue;
+  if (stages < 2 || bstages < 2) return cudaErrorInvalidValue;
   P.stages = stages;
+  P.bstages = bstages;
   P.ring = ring_depth;
-  const size_t smem = fixed + static_cast<size_t>(stages) * (kABytes + b_stage);
+  const size_t smem = fixed + static_cast<size_t>(stages) * kABytes + static_cast<size_t>(bstages) * b_stage;
   switch (ev) {
-    case 1: return launch_down_ev<1>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 2: return launch_down_ev<2>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 3: return launch_down_ev<3>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 4: return launch_down_ev<4>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 5: return launch_down_ev<5>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 6: return launch_down_ev<6>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 7: return launch_down_ev<7>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    case 8: return launch_down_ev<8>(tslot, pair, mw, sv, si, sn, P, num_sms, smem, s);
-    default: return launch_down_ev<0>(false, false, mw, sv, si, sn, P, num_sms, smem, s);
+    case 1: return launch_down_ev<1>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 2: return launch_down_ev<2>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 3: return launch_down_ev<3>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 4: return launch_down_ev<4>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 5: return launch_down_ev<5>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 6: return launch_down_ev<6>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 7: return launch_down_ev<7>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 8: return launch_down_ev<8>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    default: return launch_down_ev<0>(false, false, wide, mw, sv, si, sn, P, num_sms, smem, s);
   }
 }
 
