@@ -479,7 +479,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!valid || t >= Tn || n0 == 0) continue;
           const int base = (t << lg_tw) - col0;           // group column of in-tile index 0
-          if (n0 <= E) {
+          if (n0 <= E && base == 0 && span == tw && nsteps <= 2) {
+            // the group is exactly this tile (the common case): every slot lands
+            // in it, column bit 6 picks the K-step buffer, and the 128-byte
+            // swizzle of column c in row r is (2c mod 128) xor 16 (r mod 8)
+            int sb1 = stage0 + 1;
+            if (sb1 >= kStages) sb1 -= kStages;
+            const uint32_t row0 = smem_u32(sA + stage0 * kABytes + row_in_tile * 128);
+            const uint32_t row1 = smem_u32(sA + sb1 * kABytes + row_in_tile * 128);
+            const uint32_t rsw = row_swz << 4;
+#pragma unroll
+            for (int g = 0; g < EV; ++g) {
+              const uint32_t vw[4] = {vq[g].x, vq[g].y, vq[g].z, vq[g].w};
+              const uint32_t iw[2] = {iq[g].x, iq[g].y};
+#pragma unroll
+              for (int k2 = 0; k2 < 4; ++k2) {   // slot 8g + 2*k2 + half
+                const uint32_t cc = 2u * __byte_perm(iw[k2 >> 1], 0u, 0x4440u + 2u * (k2 & 1) + static_cast<uint32_t>(half));
+                const uint32_t addr = ((cc & 128u) ? row1 : row0) + ((cc & 127u) ^ rsw);
+                if (8 * g + 2 * k2 + half < n0) st_shared_u16(addr, half ? (vw[k2] >> 16) : vw[k2]);
+              }
+            }
+          } else if (n0 <= E) {
             const uint32_t vsh = 16u * static_cast<uint32_t>(half);   // value half of each word
 #pragma unroll
             for (int g = 0; g < EV; ++g) {
