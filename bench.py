@@ -51,17 +51,17 @@ def _kernel_source_hash(path):
         return hashlib.sha256(fh.read()).hexdigest()[:16]
 
 
-def _ncu_traffic(kernel_file, workload):
-    """DRAM bytes per launch from the committed ncu summary, only if it was taken
-    on the current source of the kernel (else null)."""
+def _ncu_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, only if it was taken on the current source of the kernel (else null)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         j = json.load(fh)
-    e = j.get(workload, {}).get(kernel_file)
+    e = j.get(workload, {}).get(kernel)
     if not e or e.get("source_sha256_16") != _kernel_source_hash(
-            os.path.join("activation_sparse_ffn_twell_b200", "csrc", kernel_file)):
+            os.path.join("activation_sparse_ffn_twell_b200", "csrc", e["source"])):
         return None
     return float(e["dram_bytes_per_launch"])
 
@@ -234,23 +234,44 @@ def run_ours(args):
     up_s = sum(up_ms) / len(up_ms) * 1e-3
     down_s = sum(down_ms) / len(down_ms) * 1e-3
     rl = _roofline_layer(L, nnz_total, touched, peaks)
-    # Per-phase rooflines.  Up: 2*M*d*f FLOP on the tensor pipe.  Down: the
-    # algorithmic work is 2*nnz*d FLOP; the tensor-core path executes the dense
-    # 2*M*d*f on h tiles rebuilt from TwELL (reported as executed_tflops).
+    # Per-phase rooflines from algorithmic work: each phase is bound by the
+    # slower of its FLOPs at the tensor peak and its unavoidable bytes at the HBM
+    # peak.  Up: 2*M*d*f FLOP (x2 gated); x + W_up (+W_gate) + b read, packed
+    # TwELL written.  Down: 2*nnz*d FLOP; the W_down rows any token touches,
+    # the packed TwELL and y.  (The tensor-core down path executes the dense
+    # 2*M*d*f on h tiles rebuilt from TwELL: reported as executed_tflops.)
+    dec_up, dec_down = _decode_paths(M, f, tw, args.mode)
+    packed = M * T_tiles * (3 * E + 2) + n_ovf * (4 + 2 * tw)
     up_flop = 2.0 * M * d * f * (2 if L.gated else 1)
+    up_bytes = 2.0 * (M * d + f * d * (2 if L.gated else 1) + f) + packed
     down_flop = 2.0 * nnz_total * d
-    phases = {
-        "up": {"kernel": "k_up_pack (fused up-GEMM + ReLU + TwELL pack, CTA pairs)",
-               "ms": up_s * 1e3, "achieved": up_flop / up_s / 1e12, "unit": "TFLOP/s",
-               "frac": up_flop / up_s / 1e12 / peaks["tc_tflops"],
-               "traffic": _ncu_traffic("k_up_pack.cu", f"relu_15b_rho{args.density:g}")},
-        "down": {"kernel": "k_spmm_mma (tensor cores on h tiles rebuilt from TwELL)"
-                           if args.mode != "gather" else "k_spmm_gather",
-                 "ms": down_s * 1e3, "achieved": down_flop / down_s / 1e12, "unit": "TFLOP/s",
-                 "frac": down_flop / down_s / 1e12 / peaks["tc_tflops"],
-                 "executed_tflops": 2.0 * M * d * f / down_s / 1e12,
-                 "traffic": _ncu_traffic("k_spmm_mma.cu", f"relu_15b_rho{args.density:g}")},
-    }
+    down_bytes = 2.0 * touched * d + packed + 2.0 * M * d
+    wkey = f"relu_15b_rho{args.density:g}" if args.workload == "relu_15b" else args.workload
+
+    def phase(kernel, desc, flop, byts, sec):
+        t_tc, t_hbm = flop / (peaks["tc_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9)
+        if t_tc >= t_hbm:
+            bound, ach, unit, peak = "tensor", flop / sec / 1e12, "TFLOP/s", peaks["tc_tflops"]
+        else:
+            bound, ach, unit, peak = "hbm", byts / sec / 1e9, "GB/s", peaks["hbm_gbs"]
+        return {"kernel": f"{kernel} ({desc})", "ms": sec * 1e3, "bound": bound, "achieved": ach,
+                "unit": unit, "peak": peak, "frac": ach / peak, "roofline_ms": max(t_tc, t_hbm) * 1e3,
+                "algorithmic_flop": flop, "algorithmic_bytes": byts,
+                "traffic": _ncu_traffic(kernel, wkey)}
+
+    if dec_up:
+        up_k = ("k_up_pack_dec", "decode batch: tokens on MMA N, ballot/prefix TwELL epilogue")
+    else:
+        up_k = ("k_up_pack", "fused up-GEMM + ReLU + TwELL pack, CTA pairs")
+    if args.mode == "gather":
+        down_k = ("k_spmm_gather", "CUDA-core gather of W_down rows per nonzero")
+    elif dec_down:
+        down_k = ("k_spmm_dec", "decode batch: split-K clusters, DSMEM reduction")
+    else:
+        down_k = ("k_spmm_mma", "tensor cores on h tiles rebuilt from TwELL")
+    phases = {"up": phase(*up_k, up_flop, up_bytes, up_s),
+              "down": phase(*down_k, down_flop, down_bytes, down_s)}
+    phases["down"]["executed_tflops"] = 2.0 * M * d * f / down_s / 1e12
     dom = max(phases, key=lambda k: phases[k]["ms"])
     P_ = phases[dom]
     result = {
@@ -264,9 +285,11 @@ def run_ours(args):
                    "tile_w": tw, "ell_w": E, "gated": bool(L.gated), "down_mode": args.mode,
                    "n_ovf": n_ovf, "l2": "flushed: 256 MiB write between timed steps",
                    "parallelism": f"token-sharded x{world} (weights replicated, no collective)"},
-        "roofline": {"bound": "tensor", "kernel": P_["kernel"], "phase": dom,
-                     "achieved": P_["achieved"], "peak": peaks["tc_tflops"], "unit": "TFLOP/s",
-                     "frac": P_["frac"], "peak_source": f"{peaks['source']} bf16 burst",
+        "roofline": {"bound": P_["bound"], "kernel": P_["kernel"], "phase": dom,
+                     "achieved": P_["achieved"], "peak": P_["peak"], "unit": P_["unit"],
+                     "frac": P_["frac"],
+                     "peak_source": f"{peaks['source']} " + ("bf16 burst" if P_["bound"] == "tensor"
+                                                              else "HBM copy"),
                      "traffic": P_["traffic"],
                      "interval": "CUDA events around the phase's C-ABI call on the launching stream"},
         "phases": phases,
@@ -275,7 +298,7 @@ def run_ours(args):
                            "useful_flop": rl["useful_flop"],
                            "unavoidable_bytes": rl["unavoidable_bytes"],
                            "touched_w_down_rows": touched, "peaks": peaks["source"]},
-        "gpu_launches": args.steps * _kernels_per_step(args.mode),
+        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down),
         "wall_s_timed_region": wall,
     }
     result["clocks"] = clk.summary()
@@ -288,8 +311,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = _cpu_baseline(L, seconds=args.cpu_seconds)
     if args.workload != "relu_15b":
-        result["note"] = ("extra workload (not the headline configuration); "
-                          "vs_baseline and the phase traffic refer to the 1.5B layer")
+        result["note"] = "extra workload (not the headline configuration)"
     if rank == 0:
         print(json.dumps(result), flush=True)
     del a
@@ -317,9 +339,18 @@ def _touched_rows(a, torch):
     return touched.sum()
 
 
-def _kernels_per_step(mode):
-    # up_pack: k_up_pack + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds k_block_path
-    # and launches both down kernels (each skips the token blocks the other owns)
+def _decode_paths(M, f, tw, mode):
+    """Which kernels the library picks (the dispatch rule of twell_up_pack and
+    twell_spmm): decode-size batches (M <= 256) use the token-on-N kernels."""
+    return (M <= 256 and tw <= 128 and f % 128 == 0), (M <= 256 and mode != "gather")
+
+
+def _kernels_per_step(mode, dec_down=False):
+    # up_pack: the producer + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds
+    # k_block_path and launches both down kernels (each skips the token blocks
+    # the other owns); the decode-size down path is one kernel
+    if dec_down:
+        return 3 + 1
     return 3 + (3 if mode == "auto" else 1)
 
 
