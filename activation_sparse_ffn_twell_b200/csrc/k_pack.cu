@@ -96,15 +96,27 @@ __global__ void __launch_bounds__(256) k_pack_dense(const uint16_t *__restrict__
 // Exclusive scan of the per-token overflow counts (one CTA, any M), total ->
 // n_ovf, capacity check -> status.
 __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
+  // each thread owns 8 consecutive rows per round of 8192 (one round up to
+  // M = 8192): two 16-byte loads, a local scan, one block scan of the totals
   __shared__ int warp_sums[32];
   __shared__ int carry_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) carry_s = 0;
-  __syncthreads();
-  for (int base = 0; base < p.M; base += 1024) {
-    const int i = base + tid;
-    const int v = (i < p.M) ? p.row_ovf[i] : 0;
-    int incl = v;
+  int carry = 0;
+  for (int base = 0; base < p.M; base += 1024 * 8) {
+    const int i0 = base + tid * 8;
+    int v[8];
+    if (i0 + 8 <= p.M) {   // the count array is 256-byte aligned: i0 * 4 is 32-byte aligned
+      const int4 a = reinterpret_cast<const int4 *>(p.row_ovf + i0)[0];
+      const int4 b = reinterpret_cast<const int4 *>(p.row_ovf + i0)[1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = (i0 + j < p.M) ? p.row_ovf[i0 + j] : 0;
+    }
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tot += v[j];
+    int incl = tot;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -120,18 +132,21 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
         if (lane >= o) ws += n;
       }
       warp_sums[lane] = ws;   // inclusive over warps
+      if (lane == 31) carry_s = ws;
     }
     __syncthreads();
-    const int carry = carry_s;
-    const int excl = carry + (warp ? warp_sums[warp - 1] : 0) + incl - v;
-    if (i < p.M) p.row_prefix[i] = excl;
-    __syncthreads();
-    if (tid == 1023) carry_s = carry + warp_sums[31];
-    __syncthreads();
+    int run = carry + (warp ? warp_sums[warp - 1] : 0) + incl - tot;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (i0 + j < p.M) p.row_prefix[i0 + j] = run;
+      run += v[j];
+    }
+    carry += carry_s;
+    __syncthreads();   // warp_sums / carry_s are rewritten by the next round
   }
   if (tid == 0) {
-    *p.n_ovf = carry_s;
-    if (carry_s > p.cap) raise_status(p.status, TWELL_ERR_OVERFLOW_CAPACITY);
+    *p.n_ovf = carry;
+    if (carry > p.cap) raise_status(p.status, TWELL_ERR_OVERFLOW_CAPACITY);
   }
 }
 

@@ -638,19 +638,31 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
   const int blk = blockIdx.x;
   const int r0 = blk * rows;
   const int nr = min(rows, A.M - r0);
-  const long long n = static_cast<long long>(nr) * A.T;
+  const int n = nr * A.T;                         // counts of the group (<= 256 x 2048)
   const uint16_t *base = A.nnz + static_cast<size_t>(r0) * A.T;
-  unsigned long long sum = 0;
-  for (long long i = threadIdx.x; i < n; i += blockDim.x) sum += __ldg(base + i);
-  __shared__ unsigned long long red[256];
-  red[threadIdx.x] = sum;
-  __syncthreads();
-  for (int o = 128; o > 0; o >>= 1) {
-    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
-    __syncthreads();
+  // the group's counts are contiguous: 16-byte loads (the group starts 16-byte
+  // aligned when rows * T is a multiple of 8), a scalar tail, 32-bit sums
+  // (at most 256 rows x 2048 tiles x 256)
+  const bool vec = ((static_cast<size_t>(r0) * A.T) & 7) == 0;
+  const int n8 = vec ? n / 8 : 0;
+  uint32_t sum = 0;
+  const uint4 *b4 = reinterpret_cast<const uint4 *>(base);
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 q = __ldg(b4 + i);
+    sum += (q.x & 0xFFFFu) + (q.x >> 16) + (q.y & 0xFFFFu) + (q.y >> 16) +
+           (q.z & 0xFFFFu) + (q.z >> 16) + (q.w & 0xFFFFu) + (q.w >> 16);
   }
+  for (int i = 8 * n8 + threadIdx.x; i < n; i += blockDim.x) sum += __ldg(base + i);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  __shared__ uint32_t red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    const double dens = static_cast<double>(red[0]) / (static_cast<double>(nr) * A.f);
+    uint32_t tot = 0;
+    for (int w = 0; w < 8; ++w) tot += red[w];
+    const double dens = static_cast<double>(tot) / (static_cast<double>(nr) * A.f);
     const int flag = dens >= crossover ? 1 : 0;
     for (int b = r0 / kBlockM; b * kBlockM < r0 + nr; ++b) blk_path[b] = flag;
   }
