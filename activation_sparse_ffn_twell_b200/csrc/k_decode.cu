@@ -364,6 +364,10 @@ __global__ void __launch_bounds__(kDecDownThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The W_down stream (warp 0) depends on no earlier kernel; every other role
+  // reads TwELL or writes y, so it waits for the previous kernels of a
+  // dependent launch here.
+  if (warp != 0) griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA: W_down tiles
@@ -712,7 +716,7 @@ cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_
 }
 
 cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y, int num_sms,
-                               cudaStream_t s) {
+                               bool pdl, cudaStream_t s) {
   if (v.M == 0) return cudaSuccess;
   DecDownParams P;
   P.A = v;
@@ -770,19 +774,8 @@ cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d
   if (encode_tensor_map_2d(&mw, w_down, d, v.f, static_cast<uint64_t>(d) * 2, 64, kBlockK,
                            CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(n_slices * best, 1, 1);
-  cfg.blockDim = dim3(kDecDownThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = best;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mw, P);
+  return launch_k(kern, dim3(n_slices * best), dim3(kDecDownThreads), smem, s, pdl,
+                  static_cast<unsigned>(best), mw, P);
 }
 
 }  // namespace twell

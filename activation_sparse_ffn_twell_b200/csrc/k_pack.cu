@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
   __shared__ int warp_sums[32];
   __shared__ int carry_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_wait();   // the producer's counts
   int carry = 0;
   for (int base = 0; base < p.M; base += 1024 * 8) {
     const int i0 = base + tid * 8;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
 // Move each staged segment to its rank in the ascending r*T+t order.
 template <int TW>
 __global__ void __launch_bounds__(256) k_ovf_scatter(PackTarget p) {
+  griddep_wait();   // the row prefix
   const int lane = threadIdx.x & 31;
   const int warps_per_cta = blockDim.x >> 5;
   const int staged = min(*p.stage_ctr, p.cap);
@@ -202,19 +204,18 @@ cudaError_t launch_pack_dense(const uint16_t *h, int ld_h, const PackTarget &t, 
 
 cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {
   if (t.M == 0) return cudaSuccess;
-  k_ovf_row_scan<<<1, 1024, 0, s>>>(t);
-  cudaError_t e = cudaGetLastError();
+  // both follow the producer kernel of the same call: dependent launches
+  cudaError_t e = launch_k(k_ovf_row_scan, dim3(1), dim3(1024), 0, s, true, 1, t);
   if (e != cudaSuccess) return e;
   if (t.cap == 0) return cudaSuccess;
-  const int grid = grid_for(t.cap, 8, 148 * 8);
+  const dim3 grid(grid_for(t.cap, 8, 148 * 8)), block(256);
   switch (t.tw) {
-    case 32: k_ovf_scatter<32><<<grid, 256, 0, s>>>(t); break;
-    case 64: k_ovf_scatter<64><<<grid, 256, 0, s>>>(t); break;
-    case 128: k_ovf_scatter<128><<<grid, 256, 0, s>>>(t); break;
-    case 256: k_ovf_scatter<256><<<grid, 256, 0, s>>>(t); break;
+    case 32: return launch_k(k_ovf_scatter<32>, grid, block, 0, s, true, 1, t);
+    case 64: return launch_k(k_ovf_scatter<64>, grid, block, 0, s, true, 1, t);
+    case 128: return launch_k(k_ovf_scatter<128>, grid, block, 0, s, true, 1, t);
+    case 256: return launch_k(k_ovf_scatter<256>, grid, block, 0, s, true, 1, t);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace twell

@@ -38,6 +38,7 @@ template <int NCH>
 __global__ void __launch_bounds__(256) k_spmm_gather(TwellView A, const uint16_t *__restrict__ W,
                                                      int d, uint16_t *__restrict__ y,
                                                      const int32_t *__restrict__ blk_path) {
+  griddep_wait();   // TwELL and the block paths of the previous kernels
   const int lane = threadIdx.x & 31;
   const int warps_per_cta = blockDim.x >> 5;
   const int cols_per_pass = 256 * NCH;
@@ -123,7 +124,7 @@ __global__ void __launch_bounds__(256) k_spmm_gather(TwellView A, const uint16_t
 }  // namespace
 
 cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                               const int32_t *blk_path, cudaStream_t s) {
+                               const int32_t *blk_path, bool pdl, cudaStream_t s) {
   if (v.M == 0) return cudaSuccess;
   // widest register tile that keeps every lane busy
   const int nch = (d >= 2048) ? 8 : (d >= 1024) ? 4 : (d >= 512) ? 2 : 1;
@@ -132,13 +133,13 @@ cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d
   long long grid = (items + 7) / 8;
   if (grid > 148 * 32) grid = 148 * 32;
   if (grid < 1) grid = 1;
+  const dim3 g(static_cast<unsigned>(grid)), b(256);
   switch (nch) {
-    case 8: k_spmm_gather<8><<<static_cast<int>(grid), 256, 0, s>>>(v, w_down, d, y, blk_path); break;
-    case 4: k_spmm_gather<4><<<static_cast<int>(grid), 256, 0, s>>>(v, w_down, d, y, blk_path); break;
-    case 2: k_spmm_gather<2><<<static_cast<int>(grid), 256, 0, s>>>(v, w_down, d, y, blk_path); break;
-    default: k_spmm_gather<1><<<static_cast<int>(grid), 256, 0, s>>>(v, w_down, d, y, blk_path); break;
+    case 8: return launch_k(k_spmm_gather<8>, g, b, 0, s, pdl, 1, v, w_down, d, y, blk_path);
+    case 4: return launch_k(k_spmm_gather<4>, g, b, 0, s, pdl, 1, v, w_down, d, y, blk_path);
+    case 2: return launch_k(k_spmm_gather<2>, g, b, 0, s, pdl, 1, v, w_down, d, y, blk_path);
+    default: return launch_k(k_spmm_gather<1>, g, b, 0, s, pdl, 1, v, w_down, d, y, blk_path);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace twell

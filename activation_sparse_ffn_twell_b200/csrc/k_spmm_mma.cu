@@ -147,6 +147,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (PAIR) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above and the W_down stream (warp 0) depend on no earlier kernel;
+  // every other role reads TwELL or writes y, so it waits for the previous
+  // kernels of a dependent launch here.
+  if (warp != 0) griddep_wait();
   const int num_tiles = P.num_m_blocks * P.num_n_blocks;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
@@ -635,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // for each 128-token block of the group so both down kernels read one array.
 __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover, int rows,
                                                     int32_t *blk_path) {
+  griddep_wait();   // the counts of the TwELL producer
   const int blk = blockIdx.x;
   const int r0 = blk * rows;
   const int nr = min(rows, A.M - r0);
@@ -671,57 +676,58 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
 template <int EV, bool TSLOT, bool PAIR, bool WIDE = false>
 cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUtensorMap &si,
                         const CUtensorMap &sn, const DownParams &P, int num_sms, size_t smem,
-                        cudaStream_t s) {
+                        bool pdl, cudaStream_t s) {
   auto kern = k_spmm_mma<EV, TSLOT, PAIR, WIDE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int tiles = P.num_m_blocks * P.num_n_blocks;
   if constexpr (PAIR) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     // persistent static schedule: only as many pairs as can be resident at once
-    cfg.gridDim = dim3(num_sms & ~1, 1, 1);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms / 2;
-    int pairs = n < num_sms / 2 ? n : num_sms / 2;
+    static int max_pairs = 0;
+    if (max_pairs == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cfg.gridDim = dim3(num_sms & ~1, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms / 2;
+      max_pairs = n;
+    }
+    int pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
     if (pairs > tiles) pairs = tiles;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    return cudaLaunchKernelEx(&cfg, kern, mw, sv, si, sn, P);
+    return launch_k(kern, dim3(2 * pairs), dim3(kThreads), smem, s, pdl, 2, mw, sv, si, sn, P);
   } else {
     const int grid = tiles < num_sms ? tiles : num_sms;
-    kern<<<grid, kThreads, smem, s>>>(mw, sv, si, sn, P);
-    return cudaGetLastError();
+    return launch_k(kern, dim3(grid), dim3(kThreads), smem, s, pdl, 1, mw, sv, si, sn, P);
   }
 }
 
 template <int EV>
 cudaError_t launch_down_ev(bool tslot, bool pair, bool wide, const CUtensorMap &mw, const CUtensorMap &sv,
                            const CUtensorMap &si, const CUtensorMap &sn, const DownParams &P,
-                           int num_sms, size_t smem, cudaStream_t s) {
+                           int num_sms, size_t smem, bool pdl, cudaStream_t s) {
   if (wide) {
     if constexpr (EV > 0) {
-      if (tslot) return launch_down<EV, true, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+      if (tslot) return launch_down<EV, true, false, true>(mw, sv, si, sn, P, num_sms, smem, pdl, s);
     }
-    return launch_down<EV, false, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+    return launch_down<EV, false, false, true>(mw, sv, si, sn, P, num_sms, smem, pdl, s);
   }
   if constexpr (EV > 0) {
     if (pair) {
-      return tslot ? launch_down<EV, true, true>(mw, sv, si, sn, P, num_sms, smem, s)
-                   : launch_down<EV, false, true>(mw, sv, si, sn, P, num_sms, smem, s);
+      return tslot ? launch_down<EV, true, true>(mw, sv, si, sn, P, num_sms, smem, pdl, s)
+                   : launch_down<EV, false, true>(mw, sv, si, sn, P, num_sms, smem, pdl, s);
     }
-    if (tslot) return launch_down<EV, true, false>(mw, sv, si, sn, P, num_sms, smem, s);
+    if (tslot) return launch_down<EV, true, false>(mw, sv, si, sn, P, num_sms, smem, pdl, s);
   }
-  return launch_down<EV, false, false>(mw, sv, si, sn, P, num_sms, smem, s);
+  return launch_down<EV, false, false>(mw, sv, si, sn, P, num_sms, smem, pdl, s);
 }
 
 }  // namespace
@@ -749,16 +755,16 @@ bool down_uses_wide() {
   return env == 1;
 }
 
-cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s) {
+cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, bool pdl,
+                              cudaStream_t s) {
   const int rows = down_uses_pair(v) ? 2 * kBlockM : kBlockM;
   const int blocks = (v.M + rows - 1) / rows;
   if (blocks == 0) return cudaSuccess;
-  k_block_path<<<blocks, 256, 0, s>>>(v, crossover, rows, blk_path);
-  return cudaGetLastError();
+  return launch_k(k_block_path, dim3(blocks), dim3(256), 0, s, pdl, 1, v, crossover, rows, blk_path);
 }
 
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                            const int32_t *blk_path, int num_sms, cudaStream_t s) {
+                            const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s) {
   if (v.M == 0) return cudaSuccess;
   CUtensorMap mw;
   if (encode_tensor_map_2d(&mw, w_down, d, v.f, static_cast<uint64_t>(d) * 2, 64, kBlockK,
@@ -826,15 +832,15 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   P.ring = ring_depth;
   const size_t smem = fixed + static_cast<size_t>(stages) * kABytes + static_cast<size_t>(bstages) * b_stage;
   switch (ev) {
-    case 1: return launch_down_ev<1>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 2: return launch_down_ev<2>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 3: return launch_down_ev<3>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 4: return launch_down_ev<4>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 5: return launch_down_ev<5>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 6: return launch_down_ev<6>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 7: return launch_down_ev<7>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    case 8: return launch_down_ev<8>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, s);
-    default: return launch_down_ev<0>(false, false, wide, mw, sv, si, sn, P, num_sms, smem, s);
+    case 1: return launch_down_ev<1>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 2: return launch_down_ev<2>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 3: return launch_down_ev<3>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 4: return launch_down_ev<4>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 5: return launch_down_ev<5>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 6: return launch_down_ev<6>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 7: return launch_down_ev<7>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    case 8: return launch_down_ev<8>(tslot, pair, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
+    default: return launch_down_ev<0>(false, false, wide, mw, sv, si, sn, P, num_sms, smem, pdl, s);
   }
 }
 

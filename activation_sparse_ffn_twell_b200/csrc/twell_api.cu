@@ -8,7 +8,8 @@
 
 namespace twell {
 
-cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, cudaStream_t s);
+cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, bool pdl,
+                              cudaStream_t s);
 
 namespace {
 
@@ -180,23 +181,29 @@ twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_
   return check_ws(ws, ws_bytes, a->M, a->tile_w, a->ovf_capacity);
 }
 
+// pdl_first: the call's first kernel may be a dependent launch (true only when
+// the previous kernel on the stream is this library's own, as in
+// twell_ffn_forward).  The later kernels of the call always are.
 twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
-                          int mode, void *ws, cudaStream_t s) {
+                          int mode, void *ws, bool pdl_first, cudaStream_t s) {
   if (a->M == 0) return TWELL_OK;
   const TwellView v = make_view(a);
   const int sms = sm_count();
   if (sms <= 0) return TWELL_ERR_CUDA;
-  if (mode == TWELL_DOWN_GATHER) return from_cuda(launch_spmm_gather(v, W_down, d_model, y, nullptr, s));
+  if (mode == TWELL_DOWN_GATHER)
+    return from_cuda(launch_spmm_gather(v, W_down, d_model, y, nullptr, pdl_first, s));
   // decode-size batches: the split-K tensor-core kernel streams W_down over every SM
-  if (decode_down_eligible(a->M)) return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, s));
-  if (mode == TWELL_DOWN_MMA) return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, s));
+  if (decode_down_eligible(a->M))
+    return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, pdl_first, s));
+  if (mode == TWELL_DOWN_MMA)
+    return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, pdl_first, s));
   const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
-  cudaError_t e = launch_block_path(v, kDownCrossoverDensity, blk, s);
+  cudaError_t e = launch_block_path(v, kDownCrossoverDensity, blk, pdl_first, s);
   if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  e = launch_spmm_gather(v, W_down, d_model, y, blk, s);
+  e = launch_spmm_gather(v, W_down, d_model, y, blk, true, s);
   if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sms, s));
+  return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sms, true, s));
 }
 
 }  // namespace
@@ -277,7 +284,7 @@ twell_status twell_spmm(const twell_matrix *a, const uint16_t *W_down, int d_mod
                         int mode, void *ws, size_t ws_bytes, void *stream) {
   twell_status st = validate_spmm(a, W_down, d_model, y, mode, ws, ws_bytes);
   if (st != TWELL_OK) return st;
-  return spmm_checked(a, W_down, d_model, y, mode, ws, static_cast<cudaStream_t>(stream));
+  return spmm_checked(a, W_down, d_model, y, mode, ws, false, static_cast<cudaStream_t>(stream));
 }
 
 twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
@@ -293,7 +300,8 @@ twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const ui
   st = up_pack_checked(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, twell, nullptr, ws,
                        ws_bytes, s);
   if (st != TWELL_OK) return st;
-  return spmm_checked(twell, W_down, d_model, y, mode, ws, s);
+  // the down kernels follow this call's own producer: dependent launches throughout
+  return spmm_checked(twell, W_down, d_model, y, mode, ws, true, s);
 }
 
 twell_status twell_read_status(const twell_matrix *a, void *stream, int32_t *n_ovf_out) {

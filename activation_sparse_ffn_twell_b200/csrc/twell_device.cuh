@@ -38,6 +38,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Wait until the grids this one depends on (programmatic dependent launch) have
+// completed and their writes are visible; a no-op when launched without it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Record an asynchronous error in the caller's status word (first error wins).
 __device__ __forceinline__ void raise_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, 0, code);

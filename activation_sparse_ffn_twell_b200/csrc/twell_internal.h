@@ -72,6 +72,39 @@ inline WsLayout ws_layout(int M, int tile_w, int cap) {
   return L;
 }
 
+// Launch `kern` on stream `s` through cudaLaunchKernelEx.  With `pdl` the grid
+// may be scheduled while the previous kernel on the stream is still finishing
+// (programmatic dependent launch): the kernel then runs griddep_wait() before it
+// touches that kernel's results.  Only launches whose predecessor is known --
+// the library's own previous kernel of the same call -- set it.  `cluster` > 1
+// groups CTAs along x into clusters of that size.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     bool pdl, unsigned cluster, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // Launchers (defined next to their kernels).  Each returns cudaSuccess or the
 // launch error; none synchronises.
@@ -89,9 +122,9 @@ cudaError_t launch_up_pack(const UpArgs &a, const PackTarget &t, int num_sms, cu
 // blk_path: NULL (the kernel owns every token block) or one int per 128-token
 // block: 0 = gather path owns it, 1 = tensor-core path owns it.
 cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                               const int32_t *blk_path, cudaStream_t s);
+                               const int32_t *blk_path, bool pdl, cudaStream_t s);
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                            const int32_t *blk_path, int num_sms, cudaStream_t s);
+                            const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s);
 
 // Decode-size batches (M <= 256): tokens on the MMA N side, weights streamed
 // over all SMs (up: one CTA per 128 hidden units; down: split-K clusters).
@@ -99,7 +132,7 @@ bool decode_up_eligible(int M, int d_ff, int tile_w);
 bool decode_down_eligible(int M);
 cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
 cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                               int num_sms, cudaStream_t s);
+                               int num_sms, bool pdl, cudaStream_t s);
 
 // Density (nonzeros / (rows * d_ff)) of a 128-token block at or above which the
 // AUTO down-projection uses the tensor-core path.  Chosen from measurement.
