@@ -58,6 +58,7 @@ __all__ = [
     "ffn_forward",
     "dense_ffn",
     "ell_width_p99",
+    "activation_stats",
 ]
 
 
@@ -218,6 +219,19 @@ def ffn_forward(x_bits, w_up_bits, b_bits, w_down_bits, tile_w, ell_w, w_gate_bi
 def dense_ffn(x_bits, w_up_bits, b_bits, w_down_bits, w_gate_bits=None) -> np.ndarray:
     """The same layer with no packing at all: bf16(h) @ W_down in float64."""
     return hidden(x_bits, w_up_bits, b_bits, w_gate_bits) @ bits_to_f64(w_down_bits)
+
+
+def activation_stats(h):
+    """Per-token statistics of the hidden activations that an L1 activation
+    regulariser works with (the pages pair ReLU sparsity with an L1 penalty:
+    upppp.jp 2026-05-11, sections 「LLMフィードフォワード層の「無駄」とは何か」 and
+    「実際の性能改善」): the L1 norm sum_j |h_rj| of the token's bf16 hidden
+    values, and its number of nonzeros (bf16 value not +-0, reading R2).
+
+    h: float64 [M, d_ff] holding bf16 values.  Returns (l1 float64 [M], nnz int64 [M]).
+    """
+    h = np.asarray(h, dtype=np.float64)
+    return np.abs(h).sum(axis=1), np.count_nonzero(h, axis=1).astype(np.int64)
 
 
 def ell_width_p99(nnz, multiple: int = 8, tile_w: Optional[int] = None) -> int:

@@ -273,3 +273,56 @@ def test_ell_width_p99_closed_form():
     assert O.ell_width_p99(np.full(1000, 17)) == 24
     v = np.concatenate([np.full(99, 3), [200]])
     assert O.ell_width_p99(v) == 8                             # nearest rank 99 of 100 -> 3
+
+
+# ---------------------------------------------------------------------------
+# Per-token activation statistics (L1 norm, nonzero count)
+# ---------------------------------------------------------------------------
+def test_stats_hand_example():
+    """The sums of |h| and the nonzero counts of the hand-computed example."""
+    g = _hand()
+    h = O.hidden(_bits(g["x"]), _bits(np.eye(8)), None)
+    l1, nnz = O.activation_stats(h)
+    assert l1.tolist() == g["expected"]["l1"]
+    assert nnz.tolist() == g["expected"]["nnz_row"]
+
+
+def test_stats_gated_negative_values_by_hand():
+    """Gated layer whose h has negative entries (worked out by hand): x = [1, 2],
+    W_gate = I, b = 0 -> ReLU(g) = [1, 2]; W_up rows [-1, 0] and [0, -3] ->
+    u = [-1, -6]; h = [-1, -12]; a second token x = [-1, 5] -> ReLU(g) = [0, 5],
+    u = [1, -15] -> h = [0, -75].  So l1 = [13, 75] and nnz = [2, 1]; a sum of
+    signed values would give [-13, -75]."""
+    x = _bits([[1, 2], [-1, 5]])
+    wg = _bits(np.eye(2))
+    wu = _bits([[-1, 0], [0, -3]])
+    h = O.hidden(x, wu, None, wg)
+    assert h.tolist() == [[-1.0, -12.0], [0.0, -75.0]]
+    l1, nnz = O.activation_stats(h)
+    assert l1.tolist() == [13.0, 75.0] and nnz.tolist() == [2, 1]
+
+
+@pytest.mark.parametrize("tw,E", [(32, 4), (64, 8), (128, 16)])
+def test_stats_agree_with_the_packed_form(tw, E):
+    """nnz per token = the packed counts summed over tiles; l1 per token = the
+    sum of |slot values| (pairs within the ELL width) plus |backup segments|."""
+    L = S.small_random(37, 64, 512, tw, E, 0.15, seed=tw)
+    h = O.hidden(L.x, L.w_up, L.b)
+    l1, nnz = O.activation_stats(h)
+    a = O.twell_pack(h, tw, E)
+    assert np.array_equal(nnz, a.nnz.astype(np.int64).sum(axis=1))
+    from_slots = np.zeros(h.shape[0])
+    vals = np.abs(O.bits_to_f64(a.vals))
+    seg = dict(zip(a.ovf_pos.tolist(), np.abs(O.bits_to_f64(a.ovf_dense))))
+    T = a.nnz.shape[1]
+    for r in range(h.shape[0]):
+        parts = [seg[r * T + t].sum() if a.nnz[r, t] > E else vals[r, t].sum() for t in range(T)]
+        from_slots[r] = math.fsum(parts)
+    assert np.allclose(l1, from_slots, rtol=1e-13, atol=0)
+    assert a.n_ovf > 0   # the backup branch is exercised
+
+
+def test_stats_zero_density():
+    L = S.small_random(8, 64, 256, 64, 8, 0.0)
+    l1, nnz = O.activation_stats(O.hidden(L.x, L.w_up, L.b))
+    assert np.all(l1 == 0) and np.all(nnz == 0)
