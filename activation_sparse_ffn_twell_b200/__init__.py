@@ -23,7 +23,8 @@ from typing import Optional
 
 __all__ = [
     "TwellError", "TwELL", "lib", "library_path", "workspace_bytes",
-    "twell_pack", "twell_up_pack", "twell_spmm", "twell_ffn_forward", "read_status",
+    "twell_pack", "twell_up_pack", "twell_up_pack_stats", "twell_spmm", "twell_ffn_forward",
+    "read_status",
     "DOWN_MODES", "STATUS", "default_ovf_capacity",
 ]
 
@@ -61,6 +62,8 @@ _SIGS = {
     "twell_pack": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P, ctypes.c_size_t, _P]),
     "twell_up_pack": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P, _P,
                            ctypes.c_size_t, _P]),
+    "twell_up_pack_stats": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P,
+                                 _P, _P, ctypes.c_size_t, _P]),
     "twell_spmm": (_I, [ctypes.POINTER(_Matrix), _P, _I, _P, _I, _P, ctypes.c_size_t, _P]),
     "twell_ffn_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P,
                                _I, _P, ctypes.c_size_t, _P]),
@@ -226,6 +229,29 @@ def twell_up_pack(x, W_up, b=None, W_gate=None, *, tile_w: int, ell_w: int,
                                 ell_w, ctypes.byref(m), _ptr(z_debug), _ptr(ws), ws.numel(),
                                 _stream_handle(stream)), "twell_up_pack")
     return a
+
+
+def twell_up_pack_stats(x, W_up, b=None, W_gate=None, *, tile_w: int, ell_w: int,
+                        out: Optional[TwELL] = None, ovf_capacity: Optional[int] = None,
+                        stream=None):
+    """twell_up_pack plus per-token activation statistics.
+
+    Returns (TwELL, l1 [M] fp32 = sum of |h| per token, nnz_row [M] int32)."""
+    torch = _torch()
+    M, d = x.shape
+    f = W_up.shape[0]
+    _need_bf16("x", x); _need_bf16("W_up", W_up, (f, d)); _need_bf16("W_gate", W_gate, (f, d))
+    _need_bf16("b", b, (f,))
+    a = out or TwELL.allocate(M, f, tile_w, ell_w, ovf_capacity, device=x.device)
+    l1 = torch.empty((M,), dtype=torch.float32, device=x.device)
+    nnz_row = torch.empty((M,), dtype=torch.int32, device=x.device)
+    nb = workspace_bytes(M, d, f, tile_w, ell_w, W_gate is not None, a.ovf_capacity)
+    ws = _workspace(nb, x.device)
+    m = a.cstruct()
+    _check(_lib().twell_up_pack_stats(_ptr(x), _ptr(W_up), _ptr(W_gate), _ptr(b), M, d, f, tile_w,
+                                      ell_w, ctypes.byref(m), _ptr(l1), _ptr(nnz_row), _ptr(ws),
+                                      ws.numel(), _stream_handle(stream)), "twell_up_pack_stats")
+    return a, l1, nnz_row
 
 
 def twell_spmm(a: TwELL, W_down, mode: str = "auto", y=None, stream=None):

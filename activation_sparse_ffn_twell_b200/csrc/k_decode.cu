@@ -56,6 +56,7 @@ struct DecUpParams {
   int num_kb, num_ub, stages;
   uint32_t tmem_cols, idesc;
   float *z_debug;
+  float *l1_part;         // NULL, or [M][T]: per (token, tile) sum of |h|
   PackTarget out;
 };
 
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int *cnt_all = reinterpret_cast<int *>(tm_full + 4);    // [group][4 warps][32 tokens]
   int *ovk_all = cnt_all + kDecEpiGroups * 128;           // [group][tiles in CTA][32 tokens]
+  float *l1_all = reinterpret_cast<float *>(ovk_all + kDecEpiGroups * 128);   // [group][4 warps][32]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -178,6 +180,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
     const int grp = (warp - 2) >> 2;
     int *cnt_s = cnt_all + grp * 128;
     int *ovk_s = ovk_all + grp * 128;
+    float *l1_s = l1_all + grp * 128;
     const uint32_t bar_id = 1u + static_cast<uint32_t>(grp);
     const int q = warp & 3;                  // TMEM lane quarter
     const int li = q % WPT;                  // this warp's place inside its hidden tile
@@ -235,6 +238,24 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
           }
         }
         cnt_s[q * 32 + lane] = myc;
+        if (P.l1_part != nullptr) {
+          // this warp's sum of |h| per token: a transposed butterfly leaves the
+          // sum for token `lane` of the chunk in lane `lane` (fixed order)
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = ok ? fabsf(__uint_as_float(hb[j] << 16)) : 0.f;
+#pragma unroll
+          for (int sh = 16; sh >= 1; sh >>= 1) {
+            const bool upper = (lane & sh) != 0;
+#pragma unroll
+            for (int i = 0; i < sh; ++i) {
+              const float send = upper ? v[i] : v[i + sh];
+              const float keep = upper ? v[i + sh] : v[i];
+              v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, sh);
+            }
+          }
+          l1_s[q * 32 + lane] = v[0];
+        }
         named_bar_sync(bar_id, 128);
         // pass 2: per token (lane = token of the chunk) the tile total and the
         // nonzeros of the tile's lower warps; the tile's first warp writes nnz
@@ -252,6 +273,11 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
           if (ok && rl < P.M) {
             const size_t pair = static_cast<size_t>(rl) * T + t;
             O.nnz[pair] = static_cast<uint16_t>(tot_l);
+            if (P.l1_part != nullptr) {   // the tile's warps in order
+              float l1t = 0.f;
+              for (int w = 0; w < WPT; ++w) l1t += l1_s[(q + w) * 32 + lane];
+              P.l1_part[pair] = l1t;
+            }
             if (tot_l > E) {
               k = atomicAdd(O.stage_ctr, 1);
               atomicAdd(O.row_ovf + rl, 1);
@@ -633,9 +659,10 @@ cudaError_t launch_up_dec_impl(const UpArgs &a, const PackTarget &t, int num_sms
   P.num_kb = a.d / kBlockK;
   P.num_ub = a.f / kDecUnits;
   P.z_debug = a.z_debug;
+  P.l1_part = a.l1_part;
   P.out = t;
   const size_t stage = (GATED ? 2 : 1) * static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
-  const size_t extra = 1024 + 4096;                      // alignment slack, barriers, counts
+  const size_t extra = 1024 + 6144;                      // alignment slack, barriers, counts
   int stages = static_cast<int>((kDecSmemBudget - extra) / stage);
   if (stages > kDecMaxStages) stages = kDecMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;

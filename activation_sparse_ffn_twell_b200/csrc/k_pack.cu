@@ -179,6 +179,34 @@ __global__ void __launch_bounds__(256) k_ovf_scatter(PackTarget p) {
   }
 }
 
+// Per token: its tiles' |h| partial sums and TwELL counts added in a fixed
+// order (each lane strides the tiles, then a fixed butterfly), so the result
+// is the same on every run.
+__global__ void __launch_bounds__(256) k_stats_reduce(PackTarget p, const float *l1_part, float *l1,
+                                                      int32_t *nnz_row) {
+  griddep_wait();   // the producer's partials and counts
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  for (int r = blockIdx.x * warps + (threadIdx.x >> 5); r < p.M; r += gridDim.x * warps) {
+    const size_t base = static_cast<size_t>(r) * p.T;
+    float s = 0.f;
+    int c = 0;
+    for (int t = lane; t < p.T; t += 32) {
+      if (l1_part != nullptr) s += l1_part[base + t];
+      c += p.nnz[base + t];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+      c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+    }
+    if (lane == 0) {
+      if (l1 != nullptr) l1[r] = s;
+      if (nnz_row != nullptr) nnz_row[r] = c;
+    }
+  }
+}
+
 int grid_for(long long work_items, int per_cta, int cap_ctas) {
   long long g = (work_items + per_cta - 1) / per_cta;
   if (g < 1) g = 1;
@@ -216,6 +244,14 @@ cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {
     case 256: return launch_k(k_ovf_scatter<256>, grid, block, 0, s, true, 1, t);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_stats_reduce(const PackTarget &t, const float *l1_part, float *l1, int32_t *nnz_row,
+                                cudaStream_t s) {
+  if (t.M == 0) return cudaSuccess;
+  // follows the backup ordering of the same call: a dependent launch
+  return launch_k(k_stats_reduce, dim3(grid_for(t.M, 8, 148 * 8)), dim3(256), 0, s, true, 1, t, l1_part,
+                  l1, nnz_row);
 }
 
 }  // namespace twell

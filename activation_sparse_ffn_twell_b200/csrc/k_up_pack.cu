@@ -53,6 +53,7 @@ struct UpParams {
   int M, d, f;
   int num_m_blocks, num_n_blocks, num_kb;
   float *z_debug;
+  float *l1_part;   // NULL, or [M][T]: per (token, tile) sum of |h| in column order
   PackTarget out;
 };
 
@@ -244,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t >= O.T) break;
         const int col0 = t * TW;                 // first hidden column of the tile
         int cnt = 0;
+        float l1 = 0.f;                          // sum of |h| over the tile, column order
 #pragma unroll 1
         for (int c = 0; c < TW / 32; ++c) {
           // a: pre-activation (gate pre-activation when gated); g: up branch
@@ -281,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t hb = bf16_bits_rn(v);
               const bool nz = (hb & 0x7FFFu) != 0;
               const bool put = nz && cnt < E;
+              l1 += fabsf(__uint_as_float(hb << 16));
               if (__any_sync(0xFFFFFFFFu, put)) {   // no store issued for all-zero columns
                 if (put) my_slots[cnt] = hb | (static_cast<uint32_t>(c * 32 + j) << 16);
               }
@@ -291,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (valid) {
           const size_t pair = static_cast<size_t>(r) * O.T + t;
           O.nnz[pair] = static_cast<uint16_t>(cnt);
+          if (P.l1_part != nullptr) P.l1_part[pair] = l1;
           uint16_t *gv = O.vals + pair * E;
           uint8_t *gi = O.idx + pair * E;
           if ((E & 7) == 0) {
@@ -419,6 +423,7 @@ cudaError_t launch_up_impl(const UpArgs &a, const PackTarget &t, int num_sms, cu
   P.num_n_blocks = GATED ? t.T : (a.f + 255) / 256;
   P.num_kb = a.d / kBlockK;
   P.z_debug = a.z_debug;
+  P.l1_part = a.l1_part;
   P.out = t;
   const size_t smem = up_smem_bytes<TW, GATED, PAIR>(t.E);
   cudaError_t e = cudaFuncSetAttribute(k_up_pack<TW, GATED, PAIR>,

@@ -73,20 +73,22 @@ twell_status check_matrix(const twell_matrix *a, int M, int d_ff, int tile_w, in
 // Workspace regions: overflow staging + per-block path flags.
 struct Ws {
   WsLayout L;
-  size_t blk_path;
+  size_t blk_path;   // [M / 128 + 1] i32: down path of each 128-token block
+  size_t l1_part;    // [M][T] fp32: per (token, tile) sums of |h| (statistics)
   size_t total;
 };
 
-Ws ws_plan(int M, int tile_w, int cap) {
+Ws ws_plan(int M, int d_ff, int tile_w, int cap) {
   Ws w;
   w.L = ws_layout(M, tile_w, cap);
   w.blk_path = w.L.total;
-  w.total = align256(w.blk_path + sizeof(int32_t) * static_cast<size_t>((M + kBlockM - 1) / kBlockM + 1));
+  w.l1_part = align256(w.blk_path + sizeof(int32_t) * static_cast<size_t>((M + kBlockM - 1) / kBlockM + 1));
+  w.total = align256(w.l1_part + sizeof(float) * static_cast<size_t>(M) * (d_ff / tile_w));
   return w;
 }
 
 PackTarget make_target(const twell_matrix *a, void *ws) {
-  const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
+  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity);
   uint8_t *base = static_cast<uint8_t *>(ws);
   PackTarget t;
   t.M = a->M; t.f = a->d_ff; t.tw = a->tile_w; t.E = a->ell_w; t.T = a->d_ff / a->tile_w;
@@ -121,29 +123,36 @@ twell_status reset_for_pack(const PackTarget &t, cudaStream_t s) {
   return from_cuda(e);
 }
 
-twell_status check_ws(void *ws, size_t ws_bytes, int M, int tile_w, int cap) {
-  const Ws w = ws_plan(M, tile_w, cap);
+twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int cap) {
+  const Ws w = ws_plan(M, d_ff, tile_w, cap);
   if (ws == nullptr || !a16(ws) || ws_bytes < w.total) return TWELL_ERR_WORKSPACE;
   return TWELL_OK;
 }
 
+// l1 / nnz_row: optional per-token statistics (twell_up_pack_stats).
 twell_status up_pack_checked(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
                              const uint16_t *b, int M, int d_model, int d_ff, int tile_w, int ell_w,
                              const twell_matrix *out, float *z_debug, void *ws, size_t ws_bytes,
-                             cudaStream_t s) {
+                             cudaStream_t s, float *l1 = nullptr, int32_t *nnz_row = nullptr) {
   if (M == 0) return TWELL_OK;
   const PackTarget t = make_target(out, ws);
   const int sms = sm_count();
   if (sms <= 0) return TWELL_ERR_CUDA;
   twell_status st = reset_for_pack(t, s);
   if (st != TWELL_OK) return st;
+  const Ws w = ws_plan(M, d_ff, tile_w, out->ovf_capacity);
+  float *l1_part = (l1 != nullptr) ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.l1_part)
+                                   : nullptr;
   UpArgs a;
   a.x = x; a.w_up = W_up; a.w_gate = W_gate; a.b = b;
-  a.M = M; a.d = d_model; a.f = d_ff; a.z_debug = z_debug;
+  a.M = M; a.d = d_model; a.f = d_ff; a.z_debug = z_debug; a.l1_part = l1_part;
   cudaError_t e = decode_up_eligible(M, d_ff, tile_w) ? launch_up_pack_decode(a, t, sms, s)
                                                        : launch_up_pack(a, t, sms, s);
   if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  return from_cuda(launch_overflow_finalize(t, s));
+  e = launch_overflow_finalize(t, s);
+  if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  if (l1 == nullptr && nnz_row == nullptr) return TWELL_OK;
+  return from_cuda(launch_stats_reduce(t, l1_part, l1, nnz_row, s));
 }
 
 twell_status validate_up(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
@@ -160,7 +169,7 @@ twell_status validate_up(const uint16_t *x, const uint16_t *W_up, const uint16_t
   if (st != TWELL_OK) return st;
   if (ell_w > kMaxEllFused) return TWELL_ERR_UNSUPPORTED;
   if (W_gate != nullptr && tile_w > 128) return TWELL_ERR_UNSUPPORTED;
-  return check_ws(ws, ws_bytes, M, tile_w, out->ovf_capacity);
+  return check_ws(ws, ws_bytes, M, d_ff, tile_w, out->ovf_capacity);
 }
 
 twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
@@ -178,7 +187,7 @@ twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_
   if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y)) return TWELL_ERR_INVALID_ARG;
   if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
     return TWELL_ERR_INVALID_ARG;
-  return check_ws(ws, ws_bytes, a->M, a->tile_w, a->ovf_capacity);
+  return check_ws(ws, ws_bytes, a->M, a->d_ff, a->tile_w, a->ovf_capacity);
 }
 
 // pdl_first: the call's first kernel may be a dependent launch (true only when
@@ -197,7 +206,7 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
     return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, pdl_first, s));
   if (mode == TWELL_DOWN_MMA)
     return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, pdl_first, s));
-  const Ws w = ws_plan(a->M, a->tile_w, a->ovf_capacity);
+  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity);
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
   cudaError_t e = launch_block_path(v, kDownCrossoverDensity, blk, pdl_first, s);
   if (e != cudaSuccess) return TWELL_ERR_CUDA;
@@ -247,7 +256,7 @@ size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w
                              int ovf_capacity) {
   if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0) return 0;
   if (d_model <= 0 || d_model % 64 != 0 || (gated != 0 && gated != 1)) return 0;
-  return ws_plan(M, tile_w, ovf_capacity).total;
+  return ws_plan(M, d_ff, tile_w, ovf_capacity).total;
 }
 
 twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
@@ -258,7 +267,7 @@ twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w
   if (h == nullptr || !a16(h) || ld_h < d_ff || ld_h % 8 != 0) return TWELL_ERR_INVALID_ARG;
   st = check_matrix(out, M, d_ff, tile_w, ell_w);
   if (st != TWELL_OK) return st;
-  st = check_ws(ws, ws_bytes, M, tile_w, out->ovf_capacity);
+  st = check_ws(ws, ws_bytes, M, d_ff, tile_w, out->ovf_capacity);
   if (st != TWELL_OK) return st;
   if (M == 0) return TWELL_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -278,6 +287,18 @@ twell_status twell_up_pack(const uint16_t *x, const uint16_t *W_up, const uint16
   if (st != TWELL_OK) return st;
   return up_pack_checked(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, out, z_debug, ws,
                          ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+twell_status twell_up_pack_stats(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                                 const uint16_t *b, int M, int d_model, int d_ff, int tile_w,
+                                 int ell_w, const twell_matrix *out, float *l1, int32_t *nnz_row,
+                                 void *ws, size_t ws_bytes, void *stream) {
+  twell_status st = validate_up(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, out, nullptr,
+                                ws, ws_bytes);
+  if (st != TWELL_OK) return st;
+  if (M > 0 && (!a16(l1) || !a16(nnz_row))) return TWELL_ERR_INVALID_ARG;
+  return up_pack_checked(x, W_up, W_gate, b, M, d_model, d_ff, tile_w, ell_w, out, nullptr, ws,
+                         ws_bytes, static_cast<cudaStream_t>(stream), l1, nnz_row);
 }
 
 twell_status twell_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,

@@ -111,11 +111,17 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 // ---------------------------------------------------------------------------
 cudaError_t launch_pack_dense(const uint16_t *h, int ld_h, const PackTarget &t, cudaStream_t s);
 cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s);
+// Per token: l1[r] = sum over tiles of l1_part[r][t] and nnz_row[r] = sum of the
+// TwELL counts (either output may be NULL), in a fixed order; a dependent launch
+// after the producer's backup ordering.
+cudaError_t launch_stats_reduce(const PackTarget &t, const float *l1_part, float *l1, int32_t *nnz_row,
+                                cudaStream_t s);
 
 struct UpArgs {
   const uint16_t *x, *w_up, *w_gate, *b;
   int M, d, f;
   float *z_debug;
+  float *l1_part;   // NULL, or [M][T] fp32: per (token, tile) sum of |h| (statistics)
 };
 cudaError_t launch_up_pack(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
 

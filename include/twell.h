@@ -126,6 +126,24 @@ twell_status twell_up_pack(const uint16_t *x, const uint16_t *W_up, const uint16
                            size_t ws_bytes, void *stream);
 
 /*
+ * twell_up_pack_stats -- twell_up_pack that also returns, per token, the
+ * statistics an L1 activation regulariser works with (the pages pair ReLU
+ * sparsity with an L1 penalty: upppp.jp 2026-05-11, sections
+ * 「LLMフィードフォワード層の「無駄」とは何か」 and 「実際の性能改善」).  The sums are
+ * taken in the producer's epilogue from the bf16 hidden values it packs.
+ *   l1      [M] fp32 or NULL: sum over the token's hidden units of |h|.  fp32 sums
+ *           in a fixed order (per tile in column order, then a fixed tree over
+ *           tiles): the same on every run, within fp32 rounding of the exact sum.
+ *   nnz_row [M] int32 or NULL: the token's number of nonzero h values.
+ * Other arguments, the TwELL output and the limits as in twell_up_pack.  The
+ * workspace (twell_workspace_bytes) holds the per-(token, tile) partial sums.
+ */
+twell_status twell_up_pack_stats(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_gate,
+                                 const uint16_t *b, int M, int d_model, int d_ff, int tile_w,
+                                 int ell_w, const twell_matrix *out, float *l1, int32_t *nnz_row,
+                                 void *ws, size_t ws_bytes, void *stream);
+
+/*
  * twell_spmm -- y = h W_down reading h only from TwELL + backup.
  *   W_down [d_ff][d_model] bf16 (row j = hidden unit j's output vector)
  *   y      [M][d_model] bf16 (fp32 accumulation, one rounding at the end)

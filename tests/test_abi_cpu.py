@@ -29,6 +29,7 @@ def _declared():
 def test_header_declares_the_three_calls():
     names = _declared()
     for n in ("twell_pack", "twell_spmm", "twell_ffn_forward", "twell_up_pack",
+              "twell_up_pack_stats", "twell_pack_noalloc",
               "twell_workspace_bytes", "twell_read_status", "twell_status_string", "twell_version"):
         assert n in names
 
@@ -97,6 +98,13 @@ def test_argument_errors_are_synchronous(L):
     m4 = _matrix(tw=256, E=16)
     assert L.twell_up_pack(x, w, w, None, 256, 256, 1024, 256, 16, bp(m4), None, ws, wsb, None) == 2
     assert L.twell_up_pack(x, w, None, None, 256, 100, 1024, 128, 16, bp(m), None, ws, wsb, None) == 1
+    # statistics variant: same validation, plus its two output pointers
+    assert L.twell_up_pack_stats(x, w, None, None, 256, 256, 1024, 128, 72, bp(m3), None, None, ws,
+                                 wsb, None) == 2
+    assert L.twell_up_pack_stats(x, w, None, None, 256, 256, 1024, 128, 16, bp(m), 0x5000004, None,
+                                 ws, wsb, None) == 1                                    # misaligned l1
+    assert L.twell_up_pack_stats(x, w, None, None, 256, 256, 1024, 128, 16, bp(m), None, None, ws,
+                                 100, None) == 6                                        # workspace
     # spmm
     assert L.twell_spmm(bp(m), None, 256, 0x5000000, 0, ws, wsb, None) == 1
     assert L.twell_spmm(bp(m), w, 256, 0x5000000, 7, ws, wsb, None) == 1               # mode
