@@ -69,6 +69,7 @@ _SIGS = {
                                _I, _P, ctypes.c_size_t, _P]),
     "twell_read_status": (_I, [ctypes.POINTER(_Matrix), _P, ctypes.POINTER(ctypes.c_int32)]),
     "twell_pack_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P]),
+    "twell_selftest_bounded_wait": (_I, [_P, _P, _P]),
 }
 
 

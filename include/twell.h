@@ -190,6 +190,18 @@ twell_status twell_pack_noalloc(const uint16_t *h, int M, int d_ff, int ld_h, in
                                 int ell_w, const twell_matrix *out, void *stream);
 
 /*
+ * twell_selftest_bounded_wait -- diagnostic for the failure path.  Every wait of
+ * the tensor-core kernels on a shared-memory barrier is bounded (about 2 s of
+ * device wall clock); one that gives up records TWELL_ERR_TIMEOUT and the kernel
+ * unwinds.  This call runs that same wait on a barrier that nothing arrives on:
+ * it must give up, set *status (device int32, caller-initialised to 0) to
+ * TWELL_ERR_TIMEOUT and write the wait's duration in ns to *elapsed_ns (device
+ * u64).  Asynchronous; the kernel takes about 2 s.  The paper has no counterpart.
+ */
+twell_status twell_selftest_bounded_wait(int32_t *status, unsigned long long *elapsed_ns,
+                                         void *stream);
+
+/*
  * Synchronise `stream`, then return the matrix's device status word (TWELL_OK if
  * clean) and, if n_ovf_out is not NULL, the true overflow-pair count.
  */
