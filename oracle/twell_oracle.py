@@ -59,6 +59,8 @@ __all__ = [
     "dense_ffn",
     "ell_width_p99",
     "activation_stats",
+    "ffn_backward",
+    "twell_transpose",
 ]
 
 
@@ -232,6 +234,48 @@ def activation_stats(h):
     """
     h = np.asarray(h, dtype=np.float64)
     return np.abs(h).sum(axis=1), np.count_nonzero(h, axis=1).astype(np.int64)
+
+
+def ffn_backward(x_bits, w_up_bits, b_bits, w_down_bits, dy_bits, round_bf16: bool = True):
+    """Backward pass of the non-gated layer y = bf16(ReLU(x W_up^T + b)) W_down for
+    a given output gradient dY, through the same sparsity pattern the forward packs
+    (the pages' training kernel runs the whole backward pass on the hybrid sparse
+    form: upppp.jp 2026-05-11, section 「TwELLとカスタムCUDAカーネルが解決する課題」).
+
+    Readings (the pages give no formulas):
+      B1  the ReLU derivative is 1 where the stored h is nonzero, 0 elsewhere;
+      B2  dZ = (dY W_down^T) masked by that pattern, stored in bf16 (one rounding);
+      B3  dX = dZ W_up, dW_up = dZ^T x, db = column sums of dZ, dW_down = h^T dY,
+          each an exact sum here (float64), rounded once to bf16 on the GPU.
+    round_bf16=False keeps h and dZ unrounded: the exact gradient of the fp64
+    piecewise-linear layer, used to pin this function against finite differences.
+
+    Returns dict(dz [M, d_ff], dx [M, d], dw_up [d_ff, d], db [d_ff], dw_down [d_ff, d]),
+    all float64.
+    """
+    x = bits_to_f64(x_bits)
+    w_up = bits_to_f64(w_up_bits)
+    w_down = bits_to_f64(w_down_bits)
+    dy = bits_to_f64(dy_bits)
+    z = x @ w_up.T
+    if b_bits is not None:
+        z = z + bits_to_f64(b_bits)[None, :]
+    h = np.maximum(z, 0.0)
+    if round_bf16:
+        h = bf16_round(h)
+    mask = h != 0.0
+    dz = np.where(mask, dy @ w_down.T, 0.0)
+    if round_bf16:
+        dz = bf16_round(dz)
+    return dict(dz=dz, dx=dz @ w_up, dw_up=dz.T @ x, db=dz.sum(axis=0), dw_down=h.T @ dy)
+
+
+def twell_transpose(a: TwELL, tile_w: int, ell_w: int) -> TwELL:
+    """The same sparse matrix with rows and columns exchanged, packed as TwELL:
+    rows = hidden units, columns = tokens cut into tiles of tile_w tokens (the
+    layout the weight gradients h^T dY and dZ^T x are read from).  Requires
+    a.M % tile_w == 0."""
+    return twell_pack(twell_unpack(a).T.copy(), tile_w, ell_w)
 
 
 def ell_width_p99(nnz, multiple: int = 8, tile_w: Optional[int] = None) -> int:

@@ -326,3 +326,73 @@ def test_stats_zero_density():
     L = S.small_random(8, 64, 256, 64, 8, 0.0)
     l1, nnz = O.activation_stats(O.hidden(L.x, L.w_up, L.b))
     assert np.all(l1 == 0) and np.all(nnz == 0)
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (non-gated) and the transposed packed form
+# ---------------------------------------------------------------------------
+def test_backward_hand_example():
+    """Worked out by hand: W_up = I, b = 0, W_down rows [1, 2] and [3, 4],
+    x = [[1, -1], [2, 3]], dY = I.  h = [[1, 0], [2, 3]]; dY W_down^T =
+    [[1, 3], [2, 4]]; masked dZ = [[1, 0], [2, 4]]; dX = dZ; dW_up = dZ^T x =
+    [[5, 5], [8, 12]]; db = [3, 4]; dW_down = h^T dY = [[1, 2], [0, 3]]."""
+    g = O.ffn_backward(_bits([[1, -1], [2, 3]]), _bits(np.eye(2)), None,
+                       _bits([[1, 2], [3, 4]]), _bits(np.eye(2)))
+    assert g["dz"].tolist() == [[1, 0], [2, 4]]
+    assert g["dx"].tolist() == [[1, 0], [2, 4]]
+    assert g["dw_up"].tolist() == [[5, 5], [8, 12]]
+    assert g["db"].tolist() == [3, 4]
+    assert g["dw_down"].tolist() == [[1, 2], [0, 3]]
+
+
+def test_backward_matches_finite_differences():
+    """Unrounded gradients against central differences of the fp64 layer
+    L = sum(relu(x W_up^T + b) W_down * dY).  x W_up^T is a multiple of 1/8 and
+    b = 1/16, so every pre-activation is at least 1/16 away from the ReLU kink: a
+    step of 2^-12 never crosses it and the layer is exactly linear along each
+    perturbed coordinate."""
+    rng = np.random.default_rng(7)
+    M, d, f = 5, 6, 9
+    x = rng.integers(-3, 4, size=(M, d)).astype(np.float64) / 2
+    wu = rng.integers(-3, 4, size=(f, d)).astype(np.float64) / 4
+    b = np.full(f, 1.0 / 16)
+    z = x @ wu.T + b
+    assert np.min(np.abs(z)) >= 1.0 / 16 and np.any(z < 0) and np.any(z > 0)
+    wd = rng.integers(-2, 3, size=(f, d)).astype(np.float64)
+    dy = rng.integers(-2, 3, size=(M, d)).astype(np.float64)
+    bits = [O.f64_to_bits(v) for v in (x, wu, b, wd, dy)]
+    for v, bb in zip((x, wu, b, wd, dy), bits):
+        assert np.array_equal(O.bits_to_f64(bb), v)            # all bf16-exact
+    g = O.ffn_backward(*bits, round_bf16=False)
+
+    def loss(x_, wu_, b_, wd_):
+        return float(np.sum(np.maximum(x_ @ wu_.T + b_[None, :], 0.0) @ wd_ * dy))
+
+    eps = 2.0 ** -12
+    for name, arr, pos in (("dx", x, 0), ("dw_up", wu, 1), ("db", b, 2), ("dw_down", wd, 3)):
+        for idx in np.ndindex(arr.shape):
+            args_p = [x.copy(), wu.copy(), b.copy(), wd.copy()]
+            args_m = [x.copy(), wu.copy(), b.copy(), wd.copy()]
+            args_p[pos][idx] += eps
+            args_m[pos][idx] -= eps
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - g[name][idx]) <= 1e-9 * max(1.0, abs(fd)), (name, idx, fd, g[name][idx])
+
+
+def test_backward_dz_has_the_forward_pattern():
+    L = S.small_random(20, 32, 128, 32, 8, 0.2, seed=5)
+    dy = S.small_random(20, 32, 128, 32, 8, 0.2, seed=6).x
+    g = O.ffn_backward(L.x, L.w_up, L.b, L.w_down, dy)
+    h = O.hidden(L.x, L.w_up, L.b)
+    assert np.all(g["dz"][h == 0] == 0)                        # zero where h is zero
+
+
+@pytest.mark.parametrize("tw,E", [(32, 4), (64, 8)])
+def test_transpose_matches_numpy_transpose(tw, E):
+    L = S.small_random(128, 32, 256, 64, 8, 0.15, seed=tw)
+    h = O.hidden(L.x, L.w_up, L.b)
+    a = O.twell_pack(h, 64, 8)
+    at = O.twell_transpose(a, tw, E)
+    assert at.M == 256 and at.d_ff == 128
+    assert np.array_equal(O.twell_unpack(at), h.T)
+    assert at.n_ovf > 0 or E >= tw
