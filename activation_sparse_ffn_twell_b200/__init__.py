@@ -24,7 +24,7 @@ from typing import Optional
 __all__ = [
     "TwellError", "TwELL", "lib", "library_path", "workspace_bytes",
     "twell_pack", "twell_up_pack", "twell_up_pack_stats", "twell_spmm", "twell_ffn_forward",
-    "read_status",
+    "twell_ffn_backward", "read_status",
     "DOWN_MODES", "STATUS", "default_ovf_capacity",
 ]
 
@@ -70,6 +70,9 @@ _SIGS = {
     "twell_read_status": (_I, [ctypes.POINTER(_Matrix), _P, ctypes.POINTER(ctypes.c_int32)]),
     "twell_pack_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P]),
     "twell_selftest_bounded_wait": (_I, [_P, _P, _P]),
+    "twell_backward_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "twell_ffn_backward": (_I, [_P, _P, _P, ctypes.POINTER(_Matrix), _P, _I, _I, _I, _P, _P, _P, _P,
+                                _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -292,6 +295,37 @@ def twell_ffn_forward(x, W_up, b, W_down, *, tile_w: int, ell_w: int, W_gate=Non
                                     _ptr(ws), ws.numel(), _stream_handle(stream)),
            "twell_ffn_forward")
     return y, a
+
+
+def twell_ffn_backward(x, W_up, W_down, h: TwELL, dY, *, ell_w_t: Optional[int] = None,
+                       ovf_capacity_t: Optional[int] = None, stream=None):
+    """Backward pass of the non-gated layer through the forward's TwELL `h`.
+
+    Returns (dX [M, d] bf16, dW_up [f, d] bf16, db [f] fp32, dW_down [f, d] bf16).
+    ell_w_t / ovf_capacity_t size the internal transposed TwELL (tiles of 128
+    tokens); by default ell_w_t = the forward's ell_w and the capacity covers
+    every (unit, token tile) pair."""
+    torch = _torch()
+    M, d = x.shape
+    f = W_up.shape[0]
+    _need_bf16("x", x); _need_bf16("W_up", W_up, (f, d)); _need_bf16("W_down", W_down, (f, d))
+    _need_bf16("dY", dY, (M, d))
+    et = ell_w_t or h.ell_w
+    cap_t = ovf_capacity_t if ovf_capacity_t is not None else f * (M // 128)
+    dX = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    dW_up = torch.empty((f, d), dtype=torch.bfloat16, device=x.device)
+    dW_down = torch.empty((f, d), dtype=torch.bfloat16, device=x.device)
+    db = torch.empty((f,), dtype=torch.float32, device=x.device)
+    nb = _lib().twell_backward_workspace_bytes(M, d, f, h.tile_w, h.ell_w, h.ovf_capacity, et, cap_t)
+    if nb == 0:
+        raise TwellError(2, f"twell_ffn_backward (M={M}, d_ff={f}, tile_w={h.tile_w})")
+    ws = _workspace(nb, x.device)
+    m = h.cstruct()
+    _check(_lib().twell_ffn_backward(_ptr(x), _ptr(W_up), _ptr(W_down), ctypes.byref(m), _ptr(dY), d,
+                                     et, cap_t, _ptr(dX), _ptr(dW_up), _ptr(db), _ptr(dW_down),
+                                     _ptr(ws), ws.numel(), _stream_handle(stream)),
+           "twell_ffn_backward")
+    return dX, dW_up, db, dW_down
 
 
 def read_status(a: TwELL, stream=None):

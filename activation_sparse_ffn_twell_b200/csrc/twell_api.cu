@@ -215,6 +215,38 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
   return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sms, true, s));
 }
 
+// Workspace of twell_ffn_backward (every region 256-byte aligned).
+struct BwLayout {
+  size_t dz_vals, dz_ovf;
+  size_t t_vals[2], t_idx[2], t_nnz[2], t_nvf[2], t_pos[2], t_dense[2];   // h^T, dZ^T
+  size_t db_part, stage, spmm, total;
+  WsLayout stage_L;
+};
+
+BwLayout bw_layout(int M, int d_ff, int tile_w, int ell_w, int cap, int ell_t, int cap_t) {
+  BwLayout b;
+  const size_t T = d_ff / tile_w, Tt = M / 128, F = d_ff;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
+  b.dz_vals = take(2 * static_cast<size_t>(M) * T * ell_w);
+  b.dz_ovf = take(2 * static_cast<size_t>(cap) * tile_w);
+  for (int i = 0; i < 2; ++i) {
+    b.t_vals[i] = take(2 * F * Tt * ell_t);
+    b.t_idx[i] = take(F * Tt * ell_t);
+    b.t_nnz[i] = take(2 * F * Tt);
+    b.t_nvf[i] = take(64);
+    b.t_pos[i] = take(4 * static_cast<size_t>(cap_t));
+    b.t_dense[i] = take(2 * 128 * static_cast<size_t>(cap_t));
+  }
+  b.db_part = take(4 * F * Tt);
+  b.stage_L = ws_layout(d_ff, 128, cap_t);
+  b.stage = take(b.stage_L.total);
+  const size_t s1 = ws_plan(M, d_ff, tile_w, cap).total, s2 = ws_plan(d_ff, M, 128, cap_t).total;
+  b.spmm = take(s1 > s2 ? s1 : s2);
+  b.total = o;
+  return b;
+}
+
 }  // namespace
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
@@ -323,6 +355,89 @@ twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const ui
   if (st != TWELL_OK) return st;
   // the down kernels follow this call's own producer: dependent launches throughout
   return spmm_checked(twell, W_down, d_model, y, mode, ws, true, s);
+}
+
+size_t twell_backward_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w,
+                                      int ovf_capacity, int ell_w_t, int ovf_capacity_t) {
+  if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0 || ovf_capacity_t < 0) return 0;
+  if (d_model <= 0 || d_model % 64 != 0 || M % 128 != 0 || d_ff % 128 != 0 || tile_w > 128) return 0;
+  if (ell_w_t < 1 || ell_w_t > 128) return 0;
+  return bw_layout(M, d_ff, tile_w, ell_w, ovf_capacity, ell_w_t, ovf_capacity_t).total;
+}
+
+twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_down,
+                                const twell_matrix *h, const uint16_t *dY, int d_model, int ell_w_t,
+                                int ovf_capacity_t, uint16_t *dX, uint16_t *dW_up, float *db,
+                                uint16_t *dW_down, void *ws, size_t ws_bytes, void *stream) {
+  if (h == nullptr) return TWELL_ERR_INVALID_ARG;
+  twell_status st = check_shape(h->M, h->d_ff, h->tile_w, h->ell_w);
+  if (st != TWELL_OK) return st;
+  const int M = h->M, f = h->d_ff, tw = h->tile_w, E = h->ell_w;
+  if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
+  if (M % 128 != 0 || f % 128 != 0 || tw > 128) return TWELL_ERR_UNSUPPORTED;
+  if (ell_w_t < 1 || ell_w_t > 128 || ovf_capacity_t < 0) return TWELL_ERR_INVALID_ARG;
+  if (M == 0) return TWELL_OK;
+  st = check_matrix(h, M, f, tw, E);
+  if (st != TWELL_OK) return st;
+  const void *ptrs[] = {x, W_up, W_down, dY, dX, dW_up, db, dW_down};
+  for (const void *q : ptrs)
+    if (q == nullptr || !a16(q)) return TWELL_ERR_INVALID_ARG;
+  const BwLayout L = bw_layout(M, f, tw, E, h->ovf_capacity, ell_w_t, ovf_capacity_t);
+  if (ws == nullptr || !a16(ws) || ws_bytes < L.total) return TWELL_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = sm_count();
+  if (sms <= 0) return TWELL_ERR_CUDA;
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  void *spmm_ws = base + L.spmm;
+
+  // 1. dZ at the forward's pattern; it shares the forward's indices, counts
+  //    and backup positions
+  const TwellView hv = make_view(h);
+  uint16_t *dz_vals = reinterpret_cast<uint16_t *>(base + L.dz_vals);
+  uint16_t *dz_ovf = reinterpret_cast<uint16_t *>(base + L.dz_ovf);
+  if (launch_sddmm(hv, dY, W_down, d_model, dz_vals, dz_ovf, sms, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  twell_matrix dz = *h;
+  dz.vals = dz_vals;
+  dz.ovf_dense = dz_ovf;
+  // 2. dX = dZ W_up
+  st = spmm_checked(&dz, W_up, d_model, dX, TWELL_DOWN_AUTO, spmm_ws, true, s);
+  if (st != TWELL_OK) return st;
+
+  // 3./5. h^T and dZ^T (tiles of 128 tokens); 4./6. dW_down = h^T dY, dW_up = dZ^T x
+  const twell_matrix *src[2] = {h, &dz};
+  const uint16_t *rhs[2] = {dY, x};
+  uint16_t *outw[2] = {dW_down, dW_up};
+  for (int i = 0; i < 2; ++i) {
+    twell_matrix tm;
+    tm.M = f; tm.d_ff = M; tm.tile_w = 128; tm.ell_w = ell_w_t;
+    tm.vals = reinterpret_cast<uint16_t *>(base + L.t_vals[i]);
+    tm.idx = base + L.t_idx[i];
+    tm.nnz = reinterpret_cast<uint16_t *>(base + L.t_nnz[i]);
+    tm.ovf_capacity = ovf_capacity_t;
+    tm.n_ovf = reinterpret_cast<int32_t *>(base + L.t_nvf[i]);
+    tm.ovf_pos = reinterpret_cast<int32_t *>(base + L.t_pos[i]);
+    tm.ovf_dense = reinterpret_cast<uint16_t *>(base + L.t_dense[i]);
+    tm.status = h->status;   // asynchronous errors land in the forward matrix's word
+    PackTarget t;
+    t.M = f; t.f = M; t.tw = 128; t.E = ell_w_t; t.T = M / 128;
+    t.vals = tm.vals; t.idx = tm.idx; t.nnz = tm.nnz;
+    t.cap = ovf_capacity_t; t.n_ovf = tm.n_ovf; t.ovf_pos = tm.ovf_pos; t.ovf_dense = tm.ovf_dense;
+    t.status = h->status;
+    t.stage_ctr = reinterpret_cast<int32_t *>(base + L.stage + L.stage_L.ctr);
+    t.row_ovf = reinterpret_cast<int32_t *>(base + L.stage + L.stage_L.row_ovf);
+    t.row_prefix = reinterpret_cast<int32_t *>(base + L.stage + L.stage_L.row_prefix);
+    t.stage_pos = reinterpret_cast<int32_t *>(base + L.stage + L.stage_L.stage_pos);
+    t.stage_dense = reinterpret_cast<uint16_t *>(base + L.stage + L.stage_L.stage_dense);
+    const size_t clr = reinterpret_cast<uint8_t *>(t.row_ovf + f) - reinterpret_cast<uint8_t *>(t.stage_ctr);
+    if (cudaMemsetAsync(t.stage_ctr, 0, clr, s) != cudaSuccess) return TWELL_ERR_CUDA;
+    float *part = (i == 1) ? reinterpret_cast<float *>(base + L.db_part) : nullptr;
+    if (launch_twell_transpose(make_view(src[i]), t, part, false, s) != cudaSuccess) return TWELL_ERR_CUDA;
+    if (launch_overflow_finalize(t, s) != cudaSuccess) return TWELL_ERR_CUDA;
+    if (i == 1 && launch_stats_reduce(t, part, db, nullptr, s) != cudaSuccess) return TWELL_ERR_CUDA;
+    st = spmm_checked(&tm, rhs[i], d_model, outw[i], TWELL_DOWN_AUTO, spmm_ws, true, s);
+    if (st != TWELL_OK) return st;
+  }
+  return TWELL_OK;
 }
 
 twell_status twell_read_status(const twell_matrix *a, void *stream, int32_t *n_ovf_out) {

@@ -132,6 +132,13 @@ cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
                             const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s);
 
+// Backward pass (non-gated): dZ = (dY W_down^T) at the forward's pattern, and
+// the TwELL transpose (tiles of 128 tokens; optional per-(unit, token tile) sums).
+cudaError_t launch_sddmm(const TwellView &h, const uint16_t *dy, const uint16_t *w_down, int d,
+                         uint16_t *dz_vals, uint16_t *dz_ovf, int num_sms, cudaStream_t s);
+cudaError_t launch_twell_transpose(const TwellView &a, const PackTarget &out, float *sum_part, bool pdl,
+                                   cudaStream_t s);
+
 // Decode-size batches (M <= 256): tokens on the MMA N side, weights streamed
 // over all SMs (up: one CTA per 128 hidden units; down: split-K clusters).
 bool decode_up_eligible(int M, int d_ff, int tile_w);

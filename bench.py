@@ -322,6 +322,8 @@ def run_ours(args):
         result["e2e"] = _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world)
         if args.sweep:
             result["density_sweep"] = _sweep(T, args, dev, peaks)
+    if args.backward and not L.gated and M % 128 == 0:
+        result["backward"] = _backward(T, x, wu, b, wd, a, args, flush, stream, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = _cpu_baseline(L, seconds=args.cpu_seconds)
     if args.workload != "relu_15b":
@@ -393,6 +395,49 @@ def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):
     ms = sum(a.elapsed_time(b) for a, b in ts) / len(ts)
     return {"ms_per_step": ms, "tokens_s": x.shape[0] / (ms * 1e-3),
             "impl": "torch.matmul bf16 (cuBLAS): relu(x W_up^T + b) W_down"}
+
+
+def _backward(T, x, wu, b, wd, a, args, flush, stream, dev):
+    """Backward pass through the hybrid form (twell_ffn_backward, given the
+    forward's TwELL) next to the same-shape dense backward through cuBLAS
+    (dH = dY W_down^T, ReLU mask, dX = dZ W_up, dW_up = dZ^T x, db, dW_down = h^T dY),
+    same run, same timing (L2 flushed between steps)."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(1)
+    dy = torch.randn(x.shape, generator=g, device=dev).to(torch.bfloat16)
+    M, f = x.shape[0], wu.shape[0]
+    cap_t = max(4096, f * (M // 128) // 8)
+
+    def ours():
+        return T.twell_ffn_backward(x, wu, wd, a, dy, ovf_capacity_t=cap_t)
+
+    h = torch.relu(torch.nn.functional.linear(x, wu, b))   # the dense forward's saved h
+
+    def dense():
+        dz = torch.matmul(dy, wd.t()) * (h > 0)
+        return torch.matmul(dz, wu), torch.matmul(dz.t(), x), dz.float().sum(0), torch.matmul(h.t(), dy)
+
+    out = {}
+    for name, fn in (("ms", ours), ("dense_ms", dense)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        out[name] = sum(p.elapsed_time(q) for p, q in ts) / len(ts)
+    code, _ = T.read_status(a)
+    out["status"] = T.STATUS[code]
+    out["impl"] = ("twell_ffn_backward: SDDMM dZ on tensor cores at the forward's pattern, dX / "
+                   "dW_down / dW_up through the sparse down-projection on transposed TwELL; dense: "
+                   "torch.matmul bf16 (cuBLAS) from the dense forward's saved h")
+    out["ovf_capacity_t"] = cap_t
+    return out
 
 
 def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
@@ -553,6 +598,8 @@ def main():
     ap.add_argument("--workload", default="relu_15b", choices=WORKLOADS,
                     help="default: the 1.5B-scale layer the headline metric is quoted on")
     ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")
+    ap.add_argument("--backward", action="store_true",
+                    help="add the backward pass (twell_ffn_backward) next to a dense cuBLAS backward")
     ap.add_argument("--quick", action="store_true", help="skip dense/e2e legs (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

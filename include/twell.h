@@ -190,6 +190,36 @@ twell_status twell_pack_noalloc(const uint16_t *h, int M, int d_ff, int ld_h, in
                                 int ell_w, const twell_matrix *out, void *stream);
 
 /*
+ * twell_ffn_backward -- backward pass of the non-gated layer
+ * y = bf16(ReLU(x W_up^T + b)) W_down through the forward's hybrid sparse form:
+ * the pages' training kernel computes the whole backward pass without dense
+ * matmuls on the sparse-main plus dense-backup representation (upppp.jp
+ * 2026-05-11, section 「TwELLとカスタムCUDAカーネルが解決する課題」).
+ *   h        the forward's TwELL of this layer (twell_up_pack / twell_ffn_forward on
+ *            the same x), read only.  Its status word also receives this call's
+ *            asynchronous errors (a bounded wait that gave up, capacity below).
+ *   dY       [M][d_model] bf16: gradient of the loss with respect to y.
+ *   dX       [M][d_model] bf16 out:   dZ W_up
+ *   dW_up    [d_ff][d_model] bf16 out: dZ^T x
+ *   db       [d_ff] fp32 out:          sum over tokens of dZ
+ *   dW_down  [d_ff][d_model] bf16 out: h^T dY
+ * where dZ = (dY W_down^T) masked to the entries h packs (the ReLU derivative is
+ * taken as 1 where the stored h is nonzero), rounded once to bf16.  Products
+ * accumulate in fp32 and round once.  h^T and dZ^T are packed internally as TwELL
+ * with tiles of 128 tokens, ell_w_t slots and ovf_capacity_t backup rows (a
+ * smaller capacity than the pairs that overflow raises TWELL_ERR_OVERFLOW_CAPACITY
+ * in h's status word and leaves the weight gradients undefined).
+ * Limits: M and d_ff multiples of 128, tile_w <= 128, 1 <= ell_w_t <= 128,
+ * d_model % 64 == 0.  Workspace: twell_backward_workspace_bytes.
+ */
+size_t twell_backward_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w,
+                                      int ovf_capacity, int ell_w_t, int ovf_capacity_t);
+twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_down,
+                                const twell_matrix *h, const uint16_t *dY, int d_model, int ell_w_t,
+                                int ovf_capacity_t, uint16_t *dX, uint16_t *dW_up, float *db,
+                                uint16_t *dW_down, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * twell_selftest_bounded_wait -- diagnostic for the failure path.  Every wait of
  * the tensor-core kernels on a shared-memory barrier is bounded (about 2 s of
  * device wall clock); one that gives up records TWELL_ERR_TIMEOUT and the kernel

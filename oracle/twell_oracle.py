@@ -236,7 +236,8 @@ def activation_stats(h):
     return np.abs(h).sum(axis=1), np.count_nonzero(h, axis=1).astype(np.int64)
 
 
-def ffn_backward(x_bits, w_up_bits, b_bits, w_down_bits, dy_bits, round_bf16: bool = True):
+def ffn_backward(x_bits, w_up_bits, b_bits, w_down_bits, dy_bits, round_bf16: bool = True,
+                 h=None):
     """Backward pass of the non-gated layer y = bf16(ReLU(x W_up^T + b)) W_down for
     a given output gradient dY, through the same sparsity pattern the forward packs
     (the pages' training kernel runs the whole backward pass on the hybrid sparse
@@ -249,6 +250,8 @@ def ffn_backward(x_bits, w_up_bits, b_bits, w_down_bits, dy_bits, round_bf16: bo
           each an exact sum here (float64), rounded once to bf16 on the GPU.
     round_bf16=False keeps h and dZ unrounded: the exact gradient of the fp64
     piecewise-linear layer, used to pin this function against finite differences.
+    h (float64 holding bf16 values), if given, is taken as the forward's hidden
+    activations -- pattern and values -- instead of being recomputed from x.
 
     Returns dict(dz [M, d_ff], dx [M, d], dw_up [d_ff, d], db [d_ff], dw_down [d_ff, d]),
     all float64.
@@ -257,12 +260,14 @@ def ffn_backward(x_bits, w_up_bits, b_bits, w_down_bits, dy_bits, round_bf16: bo
     w_up = bits_to_f64(w_up_bits)
     w_down = bits_to_f64(w_down_bits)
     dy = bits_to_f64(dy_bits)
-    z = x @ w_up.T
-    if b_bits is not None:
-        z = z + bits_to_f64(b_bits)[None, :]
-    h = np.maximum(z, 0.0)
-    if round_bf16:
-        h = bf16_round(h)
+    if h is None:
+        z = x @ w_up.T
+        if b_bits is not None:
+            z = z + bits_to_f64(b_bits)[None, :]
+        h = np.maximum(z, 0.0)
+        if round_bf16:
+            h = bf16_round(h)
+    h = np.asarray(h, dtype=np.float64)
     mask = h != 0.0
     dz = np.where(mask, dy @ w_down.T, 0.0)
     if round_bf16:

@@ -105,6 +105,11 @@ def test_argument_errors_are_synchronous(L):
                                  ws, wsb, None) == 1                                    # misaligned l1
     assert L.twell_up_pack_stats(x, w, None, None, 256, 256, 1024, 128, 16, bp(m), None, None, ws,
                                  100, None) == 6                                        # workspace
+    # backward: shape limits and workspace query
+    assert L.twell_backward_workspace_bytes(200, 256, 1024, 128, 16, 100, 16, 100) == 0   # M % 128
+    assert L.twell_backward_workspace_bytes(256, 256, 1024, 256, 16, 100, 16, 100) == 0   # tile_w
+    assert L.twell_backward_workspace_bytes(256, 256, 1024, 128, 16, 100, 16, 100) > 0
+    assert L.twell_ffn_backward(x, w, w, None, x, 256, 16, 100, x, x, x, x, ws, wsb, None) == 1
     # spmm
     assert L.twell_spmm(bp(m), None, 256, 0x5000000, 0, ws, wsb, None) == 1
     assert L.twell_spmm(bp(m), w, 256, 0x5000000, 7, ws, wsb, None) == 1               # mode
