@@ -61,6 +61,8 @@ __all__ = [
     "activation_stats",
     "ffn_backward",
     "twell_transpose",
+    "token_overflow_split",
+    "token_overflow_spmm",
 ]
 
 
@@ -281,6 +283,35 @@ def twell_transpose(a: TwELL, tile_w: int, ell_w: int) -> TwELL:
     layout the weight gradients h^T dY and dZ^T x are read from).  Requires
     a.M % tile_w == 0."""
     return twell_pack(twell_unpack(a).T.copy(), tile_w, ell_w)
+
+
+def token_overflow_split(a: TwELL):
+    """Whole-token reading of the backup (the alternative to R4): a token with any
+    tile holding more than ell_w nonzeros keeps its whole hidden row, the rest keep
+    only their ELL slots.
+
+    Returns (main, tok_pos, dense): `main` is `a` with every overflowing token's
+    counts set to 0 (its slots and backup no longer used; n_ovf = 0 since the
+    remaining tokens have no overflowing pair); `tok_pos` the overflowing tokens in
+    ascending order; `dense` their rows packed with ell_w = tile_w (every nonzero of
+    a tile fits, so no backup exists)."""
+    h = twell_unpack(a)
+    tok = np.nonzero((a.nnz.astype(np.int64) > a.ell_w).any(axis=1))[0].astype(np.int32)
+    nnz = a.nnz.copy()
+    nnz[tok] = 0
+    main = TwELL(a.M, a.d_ff, a.tile_w, a.ell_w, a.vals.copy(), a.idx.copy(), nnz,
+                 np.zeros(0, np.int32), np.zeros((0, a.tile_w), np.uint16))
+    dense = twell_pack(h[tok], a.tile_w, a.tile_w)
+    return main, tok, dense
+
+
+def token_overflow_spmm(main: TwELL, tok_pos, dense: TwELL, w_down_bits) -> np.ndarray:
+    """y for the whole-token form: the ELL slots of the remaining tokens, and a
+    small dense product for the overflowing tokens' rows."""
+    y = twell_spmm(main, w_down_bits)
+    if len(tok_pos):
+        y[np.asarray(tok_pos)] = twell_unpack(dense) @ bits_to_f64(w_down_bits)
+    return y
 
 
 def ell_width_p99(nnz, multiple: int = 8, tile_w: Optional[int] = None) -> int:

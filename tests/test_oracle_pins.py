@@ -396,3 +396,36 @@ def test_transpose_matches_numpy_transpose(tw, E):
     assert at.M == 256 and at.d_ff == 128
     assert np.array_equal(O.twell_unpack(at), h.T)
     assert at.n_ovf > 0 or E >= tw
+
+
+# ---------------------------------------------------------------------------
+# Whole-token overflow form (the alternative reading of the backup)
+# ---------------------------------------------------------------------------
+def test_token_overflow_hand_example():
+    """In the hand example only token 2 has an over-full tile (tile 0, 3 > 2
+    nonzeros): it becomes the one dense row, and y is unchanged."""
+    g = _hand()
+    e = g["expected"]
+    h = O.hidden(_bits(g["x"]), _bits(np.eye(8)), None)
+    a = O.twell_pack(h, g["tile_w"], g["ell_w"])
+    main, tok, dense = O.token_overflow_split(a)
+    assert tok.tolist() == [2]
+    assert main.nnz.tolist() == [[2, 0], [1, 1], [0, 0], [0, 0]] and main.n_ovf == 0
+    assert O.twell_unpack(dense).tolist() == [e["h"][2]]
+    assert dense.n_ovf == 0
+    y = O.token_overflow_spmm(main, tok, dense, _bits(g["w_down"]))
+    assert y.tolist() == e["y"]
+
+
+@pytest.mark.parametrize("tw,E,rho", [(32, 4, 0.15), (64, 8, 0.2), (128, 16, 0.1)])
+def test_token_overflow_matches_dense_product(tw, E, rho):
+    L = S.small_random(60, 48, 512, tw, E, rho, seed=tw + 3)
+    h = O.hidden(L.x, L.w_up, L.b)
+    a = O.twell_pack(h, tw, E)
+    main, tok, dense = O.token_overflow_split(a)
+    # the overflowing tokens, straight from h: any tile with more than E nonzeros
+    per_tile = (h.reshape(h.shape[0], -1, tw) != 0).sum(axis=2)
+    assert np.array_equal(tok, np.nonzero((per_tile > E).any(axis=1))[0])
+    assert len(tok) > 0
+    y = O.token_overflow_spmm(main, tok, dense, L.w_down)
+    assert np.allclose(y, np.matmul(h, O.bits_to_f64(L.w_down)), rtol=1e-12, atol=1e-12)
