@@ -24,7 +24,7 @@ from typing import Optional
 __all__ = [
     "TwellError", "TwELL", "lib", "library_path", "workspace_bytes",
     "twell_pack", "twell_up_pack", "twell_up_pack_stats", "twell_spmm", "twell_ffn_forward",
-    "twell_ffn_backward", "read_status",
+    "twell_ffn_backward", "twell_spmm_token_overflow", "read_status",
     "DOWN_MODES", "STATUS", "default_ovf_capacity",
 ]
 
@@ -71,6 +71,9 @@ _SIGS = {
     "twell_pack_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P]),
     "twell_selftest_bounded_wait": (_I, [_P, _P, _P]),
     "twell_backward_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "twell_token_overflow_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    "twell_spmm_token_overflow": (_I, [ctypes.POINTER(_Matrix), _P, _I, _P, _I, _P, _P,
+                                       ctypes.c_size_t, _P]),
     "twell_ffn_backward": (_I, [_P, _P, _P, ctypes.POINTER(_Matrix), _P, _I, _I, _I, _P, _P, _P, _P,
                                 _P, ctypes.c_size_t, _P]),
 }
@@ -326,6 +329,27 @@ def twell_ffn_backward(x, W_up, W_down, h: TwELL, dY, *, ell_w_t: Optional[int] 
                                      _ptr(ws), ws.numel(), _stream_handle(stream)),
            "twell_ffn_backward")
     return dX, dW_up, db, dW_down
+
+
+def twell_spmm_token_overflow(a: TwELL, W_down, cap_tok: int, y=None, stream=None):
+    """y = h W_down with the whole-token reading of the backup (tokens with any
+    over-full tile run as a small dense product).  Returns (y, n_tok device int32)."""
+    torch = _torch()
+    f, d = W_down.shape
+    _need_bf16("W_down", W_down, (a.d_ff, d))
+    if y is None:
+        y = torch.empty((a.M, d), dtype=torch.bfloat16, device=W_down.device)
+    _need_bf16("y", y, (a.M, d))
+    n_tok = torch.zeros((4,), dtype=torch.int32, device=W_down.device)
+    nb = _lib().twell_token_overflow_workspace_bytes(a.M, d, a.d_ff, a.tile_w, a.ell_w, cap_tok)
+    if nb == 0:
+        raise TwellError(1, "twell_spmm_token_overflow")
+    ws = _workspace(nb, W_down.device)
+    m = a.cstruct()
+    _check(_lib().twell_spmm_token_overflow(ctypes.byref(m), _ptr(W_down), d, _ptr(y), cap_tok,
+                                            _ptr(n_tok), _ptr(ws), ws.numel(), _stream_handle(stream)),
+           "twell_spmm_token_overflow")
+    return y, n_tok[:1]
 
 
 def read_status(a: TwELL, stream=None):

@@ -246,6 +246,11 @@ cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {
   }
 }
 
+cudaError_t launch_row_scan(const PackTarget &t, bool pdl, cudaStream_t s) {
+  if (t.M == 0) return cudaSuccess;
+  return launch_k(k_ovf_row_scan, dim3(1), dim3(1024), 0, s, pdl, 1, t);
+}
+
 cudaError_t launch_stats_reduce(const PackTarget &t, const float *l1_part, float *l1, int32_t *nnz_row,
                                 cudaStream_t s) {
   if (t.M == 0) return cudaSuccess;

@@ -247,6 +247,31 @@ BwLayout bw_layout(int M, int d_ff, int tile_w, int ell_w, int cap, int ell_t, i
   return b;
 }
 
+// Workspace of twell_spmm_token_overflow (every region 256-byte aligned).
+struct TokLayout {
+  size_t flag, rank, main_nnz, tok_pos, d_vals, d_idx, d_nnz, y_dense, words, spmm, total;
+};
+
+TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int cap_tok) {
+  TokLayout L;
+  const size_t T = d_ff / tile_w;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = align256(o + bytes); return at; };
+  L.flag = take(4 * static_cast<size_t>(M));
+  L.rank = take(4 * static_cast<size_t>(M));
+  L.main_nnz = take(2 * static_cast<size_t>(M) * T);
+  L.tok_pos = take(4 * static_cast<size_t>(cap_tok));
+  L.d_vals = take(2 * static_cast<size_t>(cap_tok) * T * tile_w);
+  L.d_idx = take(static_cast<size_t>(cap_tok) * T * tile_w);
+  L.d_nnz = take(2 * static_cast<size_t>(cap_tok) * T);
+  L.y_dense = take(2 * static_cast<size_t>(cap_tok) * d_model);
+  L.words = take(64);
+  const size_t s1 = ws_plan(M, d_ff, tile_w, 0).total, s2 = ws_plan(cap_tok, d_ff, tile_w, 0).total;
+  L.spmm = take(s1 > s2 ? s1 : s2);
+  L.total = o;
+  return L;
+}
+
 }  // namespace
 
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
@@ -438,6 +463,64 @@ twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const u
     if (st != TWELL_OK) return st;
   }
   return TWELL_OK;
+}
+
+size_t twell_token_overflow_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w,
+                                            int cap_tok) {
+  if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || cap_tok < 1) return 0;
+  if (d_model <= 0 || d_model % 64 != 0) return 0;
+  return tok_layout(M, d_model, d_ff, tile_w, cap_tok).total;
+}
+
+twell_status twell_spmm_token_overflow(const twell_matrix *a, const uint16_t *W_down, int d_model,
+                                       uint16_t *y, int cap_tok, int32_t *n_tok, void *ws,
+                                       size_t ws_bytes, void *stream) {
+  if (a == nullptr || cap_tok < 1) return TWELL_ERR_INVALID_ARG;
+  twell_status st = check_shape(a->M, a->d_ff, a->tile_w, a->ell_w);
+  if (st != TWELL_OK) return st;
+  if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
+  if (a->M == 0) return TWELL_OK;
+  st = check_matrix(a, a->M, a->d_ff, a->tile_w, a->ell_w);
+  if (st != TWELL_OK) return st;
+  if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y) || !a16(n_tok))
+    return TWELL_ERR_INVALID_ARG;
+  const int M = a->M, f = a->d_ff, tw = a->tile_w;
+  const TokLayout L = tok_layout(M, d_model, f, tw, cap_tok);
+  if (ws == nullptr || !a16(ws) || ws_bytes < L.total) return TWELL_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  int32_t *words = reinterpret_cast<int32_t *>(base + L.words);   // [0] zero n_ovf, [1] n_tok
+  int32_t *ntok = n_tok != nullptr ? n_tok : words + 1;
+  if (cudaMemsetAsync(words, 0, 64, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  const TwellView av = make_view(a);
+  int32_t *flag = reinterpret_cast<int32_t *>(base + L.flag);
+  int32_t *rank = reinterpret_cast<int32_t *>(base + L.rank);
+  if (launch_tok_flags(av, flag, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  PackTarget scan = {};
+  scan.M = M; scan.row_ovf = flag; scan.row_prefix = rank; scan.n_ovf = ntok; scan.cap = cap_tok;
+  scan.status = a->status;
+  if (launch_row_scan(scan, true, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  uint16_t *main_nnz = reinterpret_cast<uint16_t *>(base + L.main_nnz);
+  int32_t *tok_pos = reinterpret_cast<int32_t *>(base + L.tok_pos);
+  twell_matrix dm;   // the overflowing tokens' rows, ell_w = tile_w
+  dm.M = cap_tok; dm.d_ff = f; dm.tile_w = tw; dm.ell_w = tw;
+  dm.vals = reinterpret_cast<uint16_t *>(base + L.d_vals);
+  dm.idx = base + L.d_idx;
+  dm.nnz = reinterpret_cast<uint16_t *>(base + L.d_nnz);
+  dm.ovf_capacity = 0; dm.n_ovf = words; dm.ovf_pos = nullptr; dm.ovf_dense = nullptr;
+  dm.status = a->status;
+  if (launch_tok_build(av, flag, rank, ntok, cap_tok, main_nnz, tok_pos, dm.vals, dm.idx, dm.nnz, s) != cudaSuccess)
+    return TWELL_ERR_CUDA;
+  twell_matrix mm = *a;   // the other tokens: their slots, no backup
+  mm.nnz = main_nnz;
+  mm.ovf_capacity = 0; mm.n_ovf = words; mm.ovf_pos = nullptr; mm.ovf_dense = nullptr;
+  void *spmm_ws = base + L.spmm;
+  st = spmm_checked(&mm, W_down, d_model, y, TWELL_DOWN_AUTO, spmm_ws, true, s);
+  if (st != TWELL_OK) return st;
+  uint16_t *y_dense = reinterpret_cast<uint16_t *>(base + L.y_dense);
+  st = spmm_checked(&dm, W_down, d_model, y_dense, TWELL_DOWN_AUTO, spmm_ws, true, s);
+  if (st != TWELL_OK) return st;
+  return from_cuda(launch_tok_scatter(ntok, cap_tok, tok_pos, y_dense, d_model, y, s));
 }
 
 twell_status twell_read_status(const twell_matrix *a, void *stream, int32_t *n_ovf_out) {

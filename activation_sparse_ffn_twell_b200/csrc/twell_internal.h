@@ -132,6 +132,18 @@ cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
                             const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s);
 
+// Exclusive scan of t.row_ovf into t.row_prefix; the total goes to *t.n_ovf
+// (TWELL_ERR_OVERFLOW_CAPACITY in t.status when above t.cap).
+cudaError_t launch_row_scan(const PackTarget &t, bool pdl, cudaStream_t s);
+
+// Whole-token overflow form built from the per-(token, tile) form.
+cudaError_t launch_tok_flags(const TwellView &a, int32_t *flag, cudaStream_t s);
+cudaError_t launch_tok_build(const TwellView &a, const int32_t *flag, const int32_t *rank, const int32_t *n_tok,
+                             int cap, uint16_t *main_nnz, int32_t *tok_pos, uint16_t *d_vals, uint8_t *d_idx,
+                             uint16_t *d_nnz, cudaStream_t s);
+cudaError_t launch_tok_scatter(const int32_t *n_tok, int cap, const int32_t *tok_pos, const uint16_t *y_dense,
+                               int d, uint16_t *y, cudaStream_t s);
+
 // Backward pass (non-gated): dZ = (dY W_down^T) at the forward's pattern, and
 // the TwELL transpose (tiles of 128 tokens; optional per-(unit, token tile) sums).
 cudaError_t launch_sddmm(const TwellView &h, const uint16_t *dy, const uint16_t *w_down, int d,

@@ -324,6 +324,8 @@ def run_ours(args):
             result["density_sweep"] = _sweep(T, args, dev, peaks)
     if args.backward and not L.gated and M % 128 == 0:
         result["backward"] = _backward(T, x, wu, b, wd, a, args, flush, stream, dev)
+    if args.token_overflow:
+        result["token_overflow"] = _token_overflow(T, a, wd, y, args, flush, stream, dev, n_ovf)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = _cpu_baseline(L, seconds=args.cpu_seconds)
     if args.workload != "relu_15b":
@@ -437,6 +439,40 @@ def _backward(T, x, wu, b, wd, a, args, flush, stream, dev):
                    "dW_down / dW_up through the sparse down-projection on transposed TwELL; dense: "
                    "torch.matmul bf16 (cuBLAS) from the dense forward's saved h")
     out["ovf_capacity_t"] = cap_t
+    return out
+
+
+def _token_overflow(T, a, wd, y, args, flush, stream, dev, n_ovf):
+    """The two readings of the dense backup on the same packed data: per (token,
+    tile) pair (the library's form) against whole tokens (twell_spmm_token_overflow:
+    tokens with any over-full tile run as a small dense product).  Backup bytes and
+    down-projection time of each."""
+    import torch
+    _, n_tok = T.twell_spmm_token_overflow(a, wd, cap_tok=a.M)
+    torch.cuda.synchronize(dev)
+    nt = int(n_tok.item())
+    cap = max(128, (nt + 127) // 128 * 128)
+    T_ = a.d_ff // a.tile_w
+    out = {"n_overflow_pairs": n_ovf, "n_overflow_tokens": nt, "cap_tok": cap,
+           "backup_bytes_pairs": n_ovf * (4 + 2 * a.tile_w),
+           "backup_bytes_tokens_dense_rows": nt * (4 + 2 * a.d_ff),
+           "backup_bytes_tokens_as_stored": nt * T_ * (3 * a.tile_w + 2) + 4 * nt}
+    for name, fn in (("ms_pairs", lambda: T.twell_spmm(a, wd, y=y)),
+                     ("ms_tokens", lambda: T.twell_spmm_token_overflow(a, wd, cap_tok=cap, y=y))):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            ts.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        out[name] = sum(p.elapsed_time(q) for p, q in ts) / len(ts)
+    code, _ = T.read_status(a)
+    out["status"] = T.STATUS[code]
     return out
 
 
@@ -598,6 +634,8 @@ def main():
     ap.add_argument("--workload", default="relu_15b", choices=WORKLOADS,
                     help="default: the 1.5B-scale layer the headline metric is quoted on")
     ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")
+    ap.add_argument("--token-overflow", action="store_true",
+                    help="add the whole-token reading of the backup next to the per-pair one")
     ap.add_argument("--backward", action="store_true",
                     help="add the backward pass (twell_ffn_backward) next to a dense cuBLAS backward")
     ap.add_argument("--quick", action="store_true", help="skip dense/e2e legs (profiling runs)")

@@ -220,6 +220,26 @@ twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const u
                                 uint16_t *dW_down, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * twell_spmm_token_overflow -- y = h W_down with the backup read the other way
+ * (the whole-token reading of "rows that overflow spill to a dense backup"): a
+ * token with any tile holding more than ell_w nonzeros is taken out of the ELL
+ * form and its whole hidden row is stored fully dense (as TwELL with
+ * ell_w = tile_w) and run as a small dense product; the other tokens use their
+ * ELL slots.  Built from the per-(token, tile) form `a` so the two readings can
+ * be compared on the same data (backup size, time).
+ *   cap_tok  rows available for overflowing tokens; more sets
+ *            TWELL_ERR_OVERFLOW_CAPACITY in a's status word (y undefined).
+ *   n_tok    device int32 or NULL: number of overflowing tokens.
+ * Other arguments as twell_spmm (AUTO down-path selection).  Workspace:
+ * twell_token_overflow_workspace_bytes.
+ */
+size_t twell_token_overflow_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w,
+                                            int cap_tok);
+twell_status twell_spmm_token_overflow(const twell_matrix *a, const uint16_t *W_down, int d_model,
+                                       uint16_t *y, int cap_tok, int32_t *n_tok, void *ws,
+                                       size_t ws_bytes, void *stream);
+
+/*
  * twell_selftest_bounded_wait -- diagnostic for the failure path.  Every wait of
  * the tensor-core kernels on a shared-memory barrier is bounded (about 2 s of
  * device wall clock); one that gives up records TWELL_ERR_TIMEOUT and the kernel
