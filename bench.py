@@ -477,36 +477,76 @@ def _token_overflow(T, a, wd, y, args, flush, stream, dev, n_ovf):
 
 
 def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
-    """End to end through the public API with host buffers: pinned x -> device,
-    the layer, y -> pinned host, every step inside the timed region."""
+    """End to end through the public API with host buffers: each step copies its
+    tokens from pinned host memory to the device, runs twell_ffn_forward and copies
+    y back to pinned host memory, all inside the timed region.  As in a serving
+    pipeline the three run on their own streams with double-buffered device x / y
+    and host y: step i+1's upload and step i-1's download overlap step i's layer
+    (stream events order every reuse of a buffer)."""
     import numpy as np
     import torch
     from activation_sparse_ffn_twell_b200 import dist as D
     xh = torch.from_numpy(L.x.view(np.int16)).view(torch.bfloat16).pin_memory()
-    yh = torch.empty((L.M, L.d_model), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(x)
+    yh = [torch.empty((L.M, L.d_model), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xd = [torch.empty_like(x) for _ in range(2)]
+    yd = [torch.empty_like(y) for _ in range(2)]
     wg = None if L.w_gate is None else torch.from_numpy(L.w_gate.view(np.int16)).view(torch.bfloat16).to(dev)
-    for _ in range(3):
-        xd.copy_(xh, non_blocking=True)
-        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg, mode=args.mode,
-                            out=a, y=y)
-        yh.copy_(y, non_blocking=True)
+    s_up, s_cmp, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def run(n):
+        done_cmp = [None, None]   # compute of the step that last used buffer j
+        done_dn = [None, None]    # download of the step that last used buffer j
+        last = None
+        for i in range(n):
+            j = i & 1
+            with torch.cuda.stream(s_up):
+                if done_cmp[j] is not None:
+                    s_up.wait_event(done_cmp[j])
+                xd[j].copy_(xh, non_blocking=True)
+                up = torch.cuda.Event()
+                up.record(s_up)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(up)
+                if done_dn[j] is not None:
+                    s_cmp.wait_event(done_dn[j])
+                T.twell_ffn_forward(xd[j], wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg,
+                                    mode=args.mode, out=a, y=yd[j], stream=s_cmp)
+                c = torch.cuda.Event()
+                c.record(s_cmp)
+                done_cmp[j] = c
+            with torch.cuda.stream(s_dn):
+                s_dn.wait_event(c)
+                yh[j].copy_(yd[j], non_blocking=True)
+                dn = torch.cuda.Event()
+                dn.record(s_dn)
+                done_dn[j] = dn
+                last = dn
+        return last
+
+    run(3)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        xd.copy_(xh, non_blocking=True)
-        T.twell_ffn_forward(xd, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg, mode=args.mode,
-                            out=a, y=y)
-        yh.copy_(y, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_up)
+    s_cmp.wait_stream(s_up)
+    s_dn.wait_stream(s_up)
+    last = run(args.steps)
+    s_dn.wait_event(last)
+    e1.record(s_dn)
     torch.cuda.synchronize(dev)
+    # the downloaded result is the layer's output for these tokens
+    T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, W_gate=wg, mode=args.mode,
+                        out=a, y=y)
+    torch.cuda.synchronize(dev)
+    if not torch.equal(yh[(args.steps - 1) & 1].view(torch.int16), y.cpu().view(torch.int16)):
+        raise SystemExit("e2e: the downloaded y differs from the device result")
     ms = e0.elapsed_time(e1) / args.steps
     ms = D.max_over_ranks(ms, dev if world > 1 else None)
     return {"value": world * L.M / (ms * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": int(L.M * L.d_model * 2),
             "d2h_bytes_per_step": int(L.M * L.d_model * 2),
-            "ms_per_step": ms, "note": "weights resident; x in / y out through pinned host memory"}
+            "ms_per_step": ms,
+            "note": ("weights resident; x in / y out through pinned host memory every step, "
+                     "upload / layer / download pipelined on three streams")}
 
 
 def _sweep(T, args, dev, peaks):
