@@ -182,12 +182,28 @@ __global__ void __launch_bounds__(kSdThreads, 1)
         const int ns = min(n, E);
         const uint8_t *ip = H.idx + pair * E;
         uint16_t *dv = P.dz_vals + pair * E;
-#pragma unroll 4
-        for (int s = 0; s < ns; ++s) {
-          const uint32_t b = bf16_bits_rn(srow[__ldg(ip + s) & (TW - 1)]);   // (indices are < tile_w)
-          dv[s] = static_cast<uint16_t>((b & 0x7FFFu) ? b : 0u);   // -0 stored as +0
+        if ((E & 7) == 0) {
+          // eight slots at a time: one 8-byte load of their indices, one 16-byte
+          // store of their values (padding slots included)
+          for (int s0 = 0; s0 < E; s0 += 8) {
+            const uint2 iq = __ldg(reinterpret_cast<const uint2 *>(ip + s0));
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t j = ((i < 4 ? iq.x : iq.y) >> (8 * (i & 3))) & (TW - 1);   // (indices are < tile_w)
+              const uint32_t b = bf16_bits_rn(srow[j]);
+              const uint32_t v = (s0 + i < ns && (b & 0x7FFFu)) ? b : 0u;              // -0 stored as +0
+              if (i & 1) w[i >> 1] |= v << 16; else w[i >> 1] = v;
+            }
+            *reinterpret_cast<uint4 *>(dv + s0) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          for (int s = 0; s < ns; ++s) {
+            const uint32_t b = bf16_bits_rn(srow[__ldg(ip + s) & (TW - 1)]);   // (indices are < tile_w)
+            dv[s] = static_cast<uint16_t>((b & 0x7FFFu) ? b : 0u);   // -0 stored as +0
+          }
+          for (int s = ns; s < E; ++s) dv[s] = 0;                    // padding slots
         }
-        for (int s = ns; s < E; ++s) dv[s] = 0;                    // padding slots
         if (n > E) {
           const int k = ovf_lower_bound(H.ovf_pos, n_ovf, static_cast<int>(pair));
           if (k < n_ovf && __ldg(H.ovf_pos + k) == static_cast<int>(pair)) {
@@ -235,10 +251,16 @@ struct TrParams {
 };
 
 __global__ void __launch_bounds__(256) k_twell_transpose(const TrParams P) {
-  __shared__ __align__(16) uint16_t D[kTrTok][kTrUnits];   // dense block [token][unit]
+  // dynamic shared memory: the dense block D [128 tokens][128 units] bf16, then
+  // per unit its output record (E values, E indices) before the vector stores
+  extern __shared__ __align__(16) uint8_t tr_smem[];
+  uint16_t (*D)[kTrUnits] = reinterpret_cast<uint16_t (*)[kTrUnits]>(tr_smem);
   griddep_wait();   // the input's writes (a dependent launch after its producer)
   const TwellView &A = P.a;
   const PackTarget &O = P.out;
+  const int E = O.E, T = O.T;
+  uint16_t *rec_v = reinterpret_cast<uint16_t *>(tr_smem + kTrTok * kTrUnits * 2);   // [128][E]
+  uint8_t *rec_i = reinterpret_cast<uint8_t *>(rec_v + kTrUnits * E);                // [128][E]
   const int tau = blockIdx.y;                     // token tile
   const int u0 = blockIdx.x * kTrUnits;           // first hidden unit
   const int tid = threadIdx.x;
@@ -272,24 +294,37 @@ __global__ void __launch_bounds__(256) k_twell_transpose(const TrParams P) {
     }
   }
   __syncthreads();
-  // --- columns: unit threads pack their column in token order
+  // --- columns: unit threads pack their column in token order into shared
+  //     memory, then store the record with 16-byte stores
   if (tid < kTrUnits) {
     const int u = u0 + tid;
     if (u < O.M) {
-      const int E = O.E, T = O.T;
       const size_t pair = static_cast<size_t>(u) * T + tau;
-      uint16_t *ov = O.vals + pair * E;
-      uint8_t *oi = O.idx + pair * E;
+      uint16_t *sv = rec_v + tid * E;
+      uint8_t *si = rec_i + tid * E;
       int cnt = 0;
       float sum = 0.f;
       for (int r = 0; r < kTrTok; ++r) {
         const uint16_t hv = D[r][tid];
         if ((hv & 0x7FFFu) == 0) continue;
         sum += __uint_as_float(static_cast<uint32_t>(hv) << 16);
-        if (cnt < E) { ov[cnt] = hv; oi[cnt] = static_cast<uint8_t>(r); }
+        if (cnt < E) { sv[cnt] = hv; si[cnt] = static_cast<uint8_t>(r); }
         ++cnt;
       }
-      for (int s = cnt; s < E; ++s) { ov[s] = 0; oi[s] = 0; }
+      for (int s = cnt; s < E; ++s) { sv[s] = 0; si[s] = 0; }
+      uint16_t *ov = O.vals + pair * E;
+      uint8_t *oi = O.idx + pair * E;
+      if ((E & 15) == 0) {            // records 16-byte aligned: vector stores
+        for (int s = 0; s < E; s += 8) *reinterpret_cast<uint4 *>(ov + s) = *reinterpret_cast<const uint4 *>(sv + s);
+        for (int s = 0; s < E; s += 16) *reinterpret_cast<uint4 *>(oi + s) = *reinterpret_cast<const uint4 *>(si + s);
+      } else if ((E & 7) == 0) {
+        for (int s = 0; s < E; s += 8) {
+          *reinterpret_cast<uint4 *>(ov + s) = *reinterpret_cast<const uint4 *>(sv + s);
+          *reinterpret_cast<uint2 *>(oi + s) = *reinterpret_cast<const uint2 *>(si + s);
+        }
+      } else {
+        for (int s = 0; s < E; ++s) { ov[s] = sv[s]; oi[s] = si[s]; }
+      }
       O.nnz[pair] = static_cast<uint16_t>(cnt);
       if (P.sum_part != nullptr) P.sum_part[pair] = sum;
       if (cnt > E) {   // stage the dense column segment for the backup ordering
@@ -298,9 +333,14 @@ __global__ void __launch_bounds__(256) k_twell_transpose(const TrParams P) {
         if (k < O.cap) {
           O.stage_pos[k] = static_cast<int32_t>(pair);
           uint16_t *dst = O.stage_dense + static_cast<size_t>(k) * kTrTok;
-          for (int r = 0; r < kTrTok; ++r) {
-            const uint16_t hv = D[r][tid];
-            dst[r] = (hv & 0x7FFFu) ? hv : 0;
+          for (int r = 0; r < kTrTok; r += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t lo = D[r + 2 * i][tid], hi = D[r + 2 * i + 1][tid];
+              w[i] = ((lo & 0x7FFFu) ? lo : 0u) | (((hi & 0x7FFFu) ? hi : 0u) << 16);
+            }
+            *reinterpret_cast<uint4 *>(dst + r) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -359,7 +399,13 @@ cudaError_t launch_twell_transpose(const TwellView &a, const PackTarget &out, fl
   P.out = out;
   P.sum_part = sum_part;
   const dim3 grid(a.f / kTrUnits, a.M / kTrTok), block(256);
-  return launch_k(k_twell_transpose, grid, block, 0, s, pdl, 1, P);
+  // D, then the staged records (E values and E indices per unit, 16-byte aligned)
+  const size_t smem = static_cast<size_t>(kTrTok) * kTrUnits * 2 +
+                      ((static_cast<size_t>(kTrUnits) * out.E * 3 + 15) & ~static_cast<size_t>(15));
+  cudaError_t e = cudaFuncSetAttribute(k_twell_transpose, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_k(k_twell_transpose, grid, block, smem, s, pdl, 1, P);
 }
 
 }  // namespace twell
