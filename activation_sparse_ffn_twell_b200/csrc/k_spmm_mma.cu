@@ -57,7 +57,28 @@ struct DownParams {
   int slot_ib;               // bytes of the index box per row (covers ell_w indices)
   int ring;                  // slot-record ring depth (2..kSlotRing)
   const int32_t *blk_path;   // NULL, or per 128-token block: 1 = this path owns it
+  // Split schedules (512-column tiles, fast builders); a chunk is the K steps
+  // of one hidden tile (one K step when tile_w = 32).
+  //   1 (split-K): fewer tiles than CTAs.  Tile t's chunks are cut into `parts`
+  //     equal ranges; CTA p * tiles + t takes range p, so the CTAs of one range
+  //     stream the same W_down rows at the same time.
+  //   2 (shared chunks): dp_tiles whole tiles in waves of `grid` (CTA c takes
+  //     tiles c, c + grid, ...; none in the current choice), then the other
+  //     tiles' chunks dealt out evenly, numbered tile-major, over the first
+  //     sk_grid CTAs: CTA c owns chunks [c U / sk_grid, (c + 1) U / sk_grid).
+  int split;                 // 0 none, 1 split-K, 2 waves + shared remainder
+  int nc, ck;                // chunks per tile, K steps per chunk
+  int tiles, parts;          // (1)
+  int dp_tiles, sk_grid;     // (2)
+  long long units;           // (2) chunks of the shared remainder
+  float *part;               // [2 * kMaxSplitCtas][128 x 512] fp32 partial tiles
+  int32_t *split_ctr;        // [kMaxSplitCtas] arrivals per shared tile
+  int grid;                  // CTAs launched
 };
+
+// fp32 partial tile in float4 units: [32-column chunk][8 float4][128 rows], so a
+// warp's 32 rows store and load 512 contiguous bytes
+constexpr int kPartF4 = kBlockM * 512 / 4;
 
 __device__ __forceinline__ int find_ovf(const int32_t *pos, int n, int key) {
   int lo = 0, hi = n - 1;
@@ -74,6 +95,83 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
   return P.blk_path == nullptr || P.blk_path[m_blk] != 0;
 }
 
+// Schedule 2's shared remainder: CTA c owns chunks [c U / G, (c + 1) U / G).
+__device__ __forceinline__ long long split_begin(int c, long long U, int G) {
+  return static_cast<long long>(c) * U / G;
+}
+__device__ __forceinline__ int split_owner(long long q, long long U, int G) {   // CTA of chunk q
+  return static_cast<int>(((q + 1) * G + U - 1) / U - 1);
+}
+
+// The CTAs that share a tile: `n` of them, the j-th (in K order) is cta(j); each
+// publishes its fp32 partial in slot(cta) and the arrivals are counted at ctr.
+struct Sharing {
+  int n, first, stride, ctr;
+  long long ts, U;     // schedule 2: the tile's first remainder chunk, remainder size
+  int G;
+  __device__ __forceinline__ Sharing(const DownParams &P, int tile) {
+    if (P.split == 1) {
+      n = P.parts; first = tile; stride = P.tiles; ctr = tile; ts = 0; U = 0; G = 0;
+    } else {
+      U = P.units; G = P.sk_grid;
+      ts = static_cast<long long>(tile - P.dp_tiles) * P.nc;
+      first = split_owner(ts, U, G);
+      n = split_owner(ts + P.nc - 1, U, G) - first + 1;
+      stride = 1; ctr = first;
+    }
+  }
+  __device__ __forceinline__ int cta(int j) const { return first + j * stride; }
+  // schedule 2: a CTA's segment in this tile is its last one when its share
+  // began at or before the tile (slot 2c + 1), else its first one (slot 2c)
+  __device__ __forceinline__ int slot(int c) const {
+    return G == 0 ? 2 * c : 2 * c + (split_begin(c, U, G) <= ts ? 1 : 0);
+  }
+};
+
+// The CTA's work as segments: tile and K steps [kb0, kb1).
+struct Sched {
+  int mode, c, G, i;
+  long long q, qe;
+  int tile, kb0, kb1;
+  __device__ __forceinline__ Sched(const DownParams &P, bool split, int unit0, int n_units) {
+    mode = split ? P.split : 0;
+    c = unit0; G = n_units; i = 0;
+    q = qe = 0;
+    if (mode == 2 && c < P.sk_grid) {
+      q = split_begin(c, P.units, P.sk_grid);
+      qe = split_begin(c + 1, P.units, P.sk_grid);
+    }
+    tile = kb0 = kb1 = 0;
+  }
+  __device__ __forceinline__ bool next(const DownParams &P) {
+    if (mode == 1) {
+      if (i++ > 0) return false;
+      tile = c % P.tiles;
+      const int p = c / P.tiles;
+      kb0 = (p * P.nc / P.parts) * P.ck;
+      kb1 = min(((p + 1) * P.nc / P.parts) * P.ck, P.num_kb);
+      return true;
+    }
+    const int whole_end = mode == 2 ? P.dp_tiles : P.num_m_blocks * P.num_n_blocks;
+    const int t = c + i * G;
+    if (t < whole_end) {
+      ++i;
+      tile = t; kb0 = 0; kb1 = P.num_kb;
+      return true;
+    }
+    if (mode != 2 || q >= qe) return false;
+    const int r = static_cast<int>(q / P.nc);
+    const long long t0 = static_cast<long long>(r) * P.nc;
+    const int c0 = static_cast<int>(q - t0);
+    const int c1 = static_cast<int>(min(qe - t0, static_cast<long long>(P.nc)));
+    tile = P.dp_tiles + r;
+    kb0 = c0 * P.ck;
+    kb1 = min(c1 * P.ck, P.num_kb);
+    q = t0 + c1;
+    return true;
+  }
+};
+
 // EV: ell_w / 8 on the fast builder path, 0 = general path.
 // TSLOT: slot records arrive by TMA into a shared-memory ring (else per-thread loads).
 // PAIR: a cluster of 2 CTAs computes a 256-token x 256-column tile with M=256
@@ -82,13 +180,15 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
 // WIDE (single CTA only): a tile is 128 tokens x 512 y columns -- both halves
 // of TMEM -- so each rebuilt A stage feeds two 256-column MMAs, from a separate
 // ring of W_down stages.  Half as many A rebuilds per FLOP, and twice the MMA
-// time to hide each one behind.
+// time to hide each one behind.  With fast builders it takes the split
+// schedules (DownParams::split).
 template <int EV, bool TSLOT, bool PAIR, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_spmm_mma(const __grid_constant__ CUtensorMap tmap_wd, const __grid_constant__ CUtensorMap tmap_sv,
                const __grid_constant__ CUtensorMap tmap_si, const __grid_constant__ CUtensorMap tmap_sn,
                const DownParams P) {
   static_assert(!(WIDE && PAIR), "512-column tiles are single-CTA");
+  constexpr bool SPLIT = WIDE && EV > 0;                      // split schedule compiled in
   constexpr int NH = WIDE ? 2 : 1;                            // 256-column halves per tile
   constexpr int kTN = NH * kBN;                               // y columns per tile
   constexpr int TILE_M = PAIR ? 2 * kBlockM : kBlockM;
@@ -114,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *bempty = bfull + kMaxStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bempty + kMaxStages);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile int *split_last = abort_flag + 1;                   // epilogue: last contributor
   // slot ring entry: [128][ell_w] bf16 values, [128][slot_ib] u8 indices, [128][8] u16 nnz
   uint8_t *sRing = reinterpret_cast<uint8_t *>(bars) + 512;
   const int ring_v = kBlockM * 2 * P.A.E, ring_i = kBlockM * P.slot_ib;
@@ -157,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int unit0 = PAIR ? static_cast<int>(cluster_id_x()) : static_cast<int>(blockIdx.x);
   const int n_units = PAIR ? static_cast<int>(num_clusters_x()) : static_cast<int>(gridDim.x);
   const int row_base = static_cast<int>(rank) * kBlockM;   // this CTA's rows inside a tile
+  const bool split = SPLIT && P.split != 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA (W_down)
@@ -164,11 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0; uint32_t phase = 0; uint32_t filled = 0;
       int bst = 0; uint32_t bph = 0; uint32_t bfilled = 0;   // W_down ring (WIDE)
       bool ok = true;
-      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
+      Sched sc(P, split, unit0, n_units);
+      while (ok && sc.next(P)) {
+        const int tile = sc.tile;
         const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         if constexpr (WIDE) {
-          for (int kb = 0; kb < P.num_kb && ok; ++kb) {
+          for (int kb = sc.kb0; kb < sc.kb1 && ok; ++kb) {
             if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
             filled |= 1u << stage;
             mbar_arrive(&full[stage]);   // (no bytes: the builders fill A)
@@ -187,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           continue;
         }
-        for (int kb = 0; kb < P.num_kb; ++kb) {
+        for (int kb = sc.kb0; kb < sc.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * B_BYTES);
           filled |= 1u << stage;
@@ -224,8 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0; uint32_t phase = 0; int it = 0;
       int bst = 0; uint32_t bph = 0;   // W_down ring (WIDE)
       bool ok = true;
-      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
-        const int m_blk = tile % P.num_m_blocks;
+      Sched sc(P, split, unit0, n_units);
+      while (ok && sc.next(P)) {
+        const int m_blk = sc.tile % P.num_m_blocks;
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         // WIDE: one accumulator set (both TMEM halves); else two, alternating
         const int acc = WIDE ? 0 : (it & 1);
@@ -235,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
         if constexpr (WIDE) {
-          for (int kb = 0; kb < P.num_kb && ok; ++kb) {
+          for (int kb = sc.kb0; kb < sc.kb1 && ok; ++kb) {
             if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t a_addr = smem_u32(sA + stage * kABytes);
@@ -247,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int k = 0; k < kBlockK / kUmmaK; ++k) {
                 const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
                 const uint64_t bdesc = smem_desc_sw128(b_addr + k * 2048, kBlockK * 128, 1024);
-                umma_bf16(d_tmem + h * kBN, adesc, bdesc, IDESC, (kb | k) != 0);
+                umma_bf16(d_tmem + h * kBN, adesc, bdesc, IDESC, (kb != sc.kb0 || k != 0));
               }
               umma_commit(&bempty[bst]);
               if (++bst == kBStages) { bst = 0; bph ^= 1u; }
@@ -259,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&tm_full[acc]);
           continue;
         }
-        for (int kb = 0; kb < P.num_kb; ++kb) {
+        for (int kb = sc.kb0; kb < sc.kb1; ++kb) {
           if (!mbar_wait<PAIR>(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(sA + stage * kABytes);
@@ -269,8 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t adesc = smem_desc_sw128(a_addr + k * 32, 16, 1024);
             // N-major B: 16 K-rows of 128 B per step; 64-column groups 8 KB apart
             const uint64_t bdesc = smem_desc_sw128(b_addr + k * 2048, kBlockK * 128, 1024);
-            if constexpr (PAIR) umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
-            else umma_bf16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0);
+            if constexpr (PAIR) umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb != sc.kb0 || k != 0));
+            else umma_bf16(d_tmem, adesc, bdesc, IDESC, (kb != sc.kb0 || k != 0));
           }
           if constexpr (PAIR) umma_commit_pair_mc(&empty[stage], 0x3);
           else umma_commit(&empty[stage]);
@@ -295,11 +400,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t bytes = static_cast<uint32_t>(ring_entry);
       int cnt = 0;
       bool ok = true;
-      for (int tile = unit0; tile < num_tiles && ok; tile += n_units) {
-        const int m_blk = tile % P.num_m_blocks;
+      Sched sc(P, split, unit0, n_units);
+      while (ok && sc.next(P)) {
+        const int m_blk = sc.tile % P.num_m_blocks;
         if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
         const int r0 = m_blk * TILE_M + row_base;
-        for (int t = 0; t < A.T; ++t, ++cnt) {
+        // the hidden tiles of the segment's K steps, in the builders' order
+        const int t0 = (sc.kb0 * kBlockK) / A.tw;
+        const int t1 = min((sc.kb1 * kBlockK + A.tw - 1) / A.tw, A.T);
+        for (int t = t0; t < t1; ++t, ++cnt) {
           const int ring = cnt % kRing;
           const uint32_t ph = static_cast<uint32_t>(cnt / kRing) & 1u;
           if (!mbar_wait(&s_empty[ring], ph ^ 1u, abort_flag)) { ok = false; break; }
@@ -322,13 +431,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int row_in_tile = q * 32 + lane;
     int it = 0;
-    for (int tile = unit0; tile < num_tiles; tile += n_units) {
+    Sched sc(P, split, unit0, n_units);
+    while (sc.next(P)) {
+      const int tile = sc.tile;
       const int m_blk = tile % P.num_m_blocks, n_blk = tile / P.num_m_blocks;
       if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
       const int acc = WIDE ? 0 : (it & 1);
       const uint32_t acc_phase = WIDE ? (it & 1) : ((it >> 1) & 1);
       ++it;
-      if (!mbar_wait<PAIR>(&tm_full[acc], acc_phase, abort_flag)) {
+      bool waited = mbar_wait<PAIR>(&tm_full[acc], acc_phase, abort_flag);
+      // one decision per warp (its TMEM loads are warp-wide); with the split
+      // schedule one for all four epilogue warps, which meet at barriers below
+      waited = __all_sync(0xFFFFFFFFu, waited);
+      if (split) waited = !named_bar_any(2, 128, !waited);
+      if (!waited) {
         *abort_flag = 1;
         raise_status(A.status, TWELL_ERR_TIMEOUT);
         break;
@@ -338,12 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool valid = r < A.M;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
       uint16_t *yr = P.y + static_cast<size_t>(r) * P.d + n_blk * kTN;
-#pragma unroll 1
-      for (int c = 0; c < kTN / 32; ++c) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(t_row + c * 32, v);
-        tmem_ld_wait();
+      constexpr int NCH = kTN / 32;   // 32-column chunks of the accumulator (8 or 16)
+      // bf16 y of chunk c from 32 fp32 words
+      auto store_y = [&](const uint32_t (&v)[32], int c) {
         if (valid && n_blk * kTN + c * 32 < P.d) {
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
@@ -354,6 +467,126 @@ __global__ void __launch_bounds__(kThreads, 1)
             o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
             *reinterpret_cast<uint4 *>(yr + c * 32 + j) = o;
           }
+        }
+      };
+      // Every chunk pass keeps the next chunk's TMEM load in flight while the
+      // current one is converted and stored.
+      auto for_chunks = [&](auto &&body) {
+        uint32_t va[32], vb[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(t_row, va);
+        tmem_ld_wait_r32(va);
+#pragma unroll 1
+        for (int c = 0; c < NCH; c += 2) {
+          __syncwarp();
+          tmem_ld_32x32b_x32(t_row + (c + 1) * 32, vb);
+          body(va, c);
+          tmem_ld_wait_r32(vb);
+          if (c + 2 < NCH) {
+            __syncwarp();
+            tmem_ld_32x32b_x32(t_row + (c + 2) * 32, va);
+          }
+          body(vb, c + 1);
+          if (c + 2 < NCH) tmem_ld_wait_r32(va);
+        }
+      };
+      if (!split || (sc.kb0 == 0 && sc.kb1 == P.num_kb)) {
+        for_chunks(store_y);
+      } else if constexpr (SPLIT) {
+        // A tile shared with other CTAs: publish this CTA's fp32 partial, count
+        // the arrival, and the last of the contributors adds all partials in K
+        // order (0 + p_0 + ... + p_n-1: the same bits whichever CTA finishes
+        // last) before the one bf16 rounding.
+        const Sharing sh(P, tile);
+        const int me = static_cast<int>(blockIdx.x);
+        float4 *part = reinterpret_cast<float4 *>(P.part);
+        float4 *mine = part + static_cast<size_t>(sh.slot(me)) * kPartF4 + row_in_tile;
+        for_chunks([&](const uint32_t (&v)[32], int c) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            __stcs(mine + (c * 8 + j) * kBlockM,   // streaming: read once, by the finishing CTA
+                   make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+        });
+        __threadfence();
+        named_bar_sync(2, 128);   // the four epilogue warps
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(P.split_ctr + sh.ctr, 1);
+          *split_last = (old == sh.n - 1) ? 1 : 0;
+        }
+        named_bar_sync(2, 128);
+        if (*split_last) {
+          __threadfence();
+          if (sh.n == 2) {
+            // Two contributors: fp32 addition is commutative, so own + other
+            // has the bits of p_0 + p_1.  The other's next chunk is in flight
+            // while the current one is added and stored.
+            const int other = sh.cta(0) == me ? sh.cta(1) : sh.cta(0);
+            const float4 *src = part + static_cast<size_t>(sh.slot(other)) * kPartF4 + row_in_tile;
+            float4 qa[8], qb[8];
+            auto add_store = [&](const uint32_t (&v)[32], const float4 (&q)[8], int c) {
+              uint32_t w[32];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                w[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + q[j].x);
+                w[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + q[j].y);
+                w[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q[j].z);
+                w[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q[j].w);
+              }
+              store_y(w, c);
+            };
+#pragma unroll
+            for (int j = 0; j < 8; ++j) qa[j] = __ldcs(src + j * kBlockM);
+#pragma unroll 1
+            for (int c = 0; c < NCH; c += 2) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) qb[j] = __ldcs(src + ((c + 1) * 8 + j) * kBlockM);
+              uint32_t v[32];
+              __syncwarp();
+              tmem_ld_32x32b_x32(t_row + c * 32, v);
+              tmem_ld_wait_r32(v);
+              add_store(v, qa, c);
+              if (c + 2 < NCH) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) qa[j] = __ldcs(src + ((c + 2) * 8 + j) * kBlockM);
+              }
+              __syncwarp();
+              tmem_ld_32x32b_x32(t_row + (c + 1) * 32, v);
+              tmem_ld_wait_r32(v);
+              add_store(v, qb, c + 1);
+            }
+          } else {
+#pragma unroll 1
+            for (int c = 0; c < NCH; ++c) {
+              float s32[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) s32[j] = 0.0f;
+              for (int jj = 0; jj < sh.n; ++jj) {
+                const int k = sh.cta(jj);
+                if (k == me) {
+                  uint32_t v[32];
+                  __syncwarp();
+                  tmem_ld_32x32b_x32(t_row + c * 32, v);
+                  tmem_ld_wait_r32(v);
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) s32[j] += __uint_as_float(v[j]);
+                } else {
+                  const float4 *src = part + static_cast<size_t>(sh.slot(k)) * kPartF4 +
+                                      static_cast<size_t>(c * 8) * kBlockM + row_in_tile;
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) {
+                    const float4 q4 = __ldcs(src + j * kBlockM);
+                    s32[4 * j] += q4.x; s32[4 * j + 1] += q4.y; s32[4 * j + 2] += q4.z; s32[4 * j + 3] += q4.w;
+                  }
+                }
+              }
+              uint32_t w[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(s32[j]);
+              store_y(w, c);
+            }
+          }
+          if (threadIdx.x == 64) P.split_ctr[sh.ctr] = 0;   // every contributor has arrived
         }
       }
       tc_fence_before();
@@ -383,8 +616,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The eight builder warps meet at a named barrier once per group of K
     // steps; a bounded wait that gives up is OR-ed into that barrier so they all
     // leave at the same group (no warp is left waiting for the others).
-    for (int tile = unit0; tile < num_tiles; tile += n_units) {
-      const int m_blk = tile % P.num_m_blocks;
+    Sched sc(P, split, unit0, n_units);
+    while (sc.next(P)) {
+      const int m_blk = sc.tile % P.num_m_blocks;
       if (!tile_owned(P, m_blk * (TILE_M / kBlockM))) continue;
       const int r = m_blk * TILE_M + row_base + row_in_tile;
       const bool valid = r < A.M;
@@ -411,8 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the ring holds them) so every slot is visited once per tile
       // (at most stages-1 of them, so the MMA always has a stage to work on)
       const int S = max(1, min(tw / kBlockK, kStages - 1));
-      for (int kb0 = 0; kb0 < P.num_kb; kb0 += S) {
-        const int nsteps = min(S, P.num_kb - kb0);
+      for (int kb0 = sc.kb0; kb0 < sc.kb1; kb0 += S) {
+        const int nsteps = min(S, sc.kb1 - kb0);
         const int stage0 = stage;
         // claim the group's A stages as soon as the MMA has released them and
         // clear this thread's half of its row (row-XOR chunk order: the 32 rows
@@ -476,7 +710,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // of the row is entry ovf_base + k
             ovf_k = -1;
             if (n0 > E) {
-              if (ovf_base < 0) ovf_base = ovf_lower_bound(A.ovf_pos, n_ovf, static_cast<int>(pair0));
+              // (first overflowing tile of the row in this segment: its own entry)
+              if (ovf_base < 0) ovf_base = ovf_lower_bound(A.ovf_pos, n_ovf, static_cast<int>(pair0) + t);
               ovf_k = ovf_base + ovf_seen++;
               if (ovf_k >= n_ovf) ovf_k = -1;   // capacity exhausted: y is undefined
             }
@@ -638,8 +873,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // pairs): 1 when its density is at or above the crossover.  The flag is written
 // for each 128-token block of the group so both down kernels read one array.
 __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover, int rows,
-                                                    int32_t *blk_path) {
+                                                    int32_t *blk_path, int32_t *split_ctr) {
   griddep_wait();   // the counts of the TwELL producer
+  // the split schedule's arrival counters start every launch at zero
+  if (split_ctr != nullptr && blockIdx.x == 0 && threadIdx.x < kMaxSplitCtas) split_ctr[threadIdx.x] = 0;
   const int blk = blockIdx.x;
   const int r0 = blk * rows;
   const int nr = min(rows, A.M - r0);
@@ -705,7 +942,7 @@ cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUte
     if (pairs > tiles) pairs = tiles;
     return launch_k(kern, dim3(2 * pairs), dim3(kThreads), smem, s, pdl, 2, mw, sv, si, sn, P);
   } else {
-    const int grid = tiles < num_sms ? tiles : num_sms;
+    const int grid = P.split ? P.grid : (tiles < num_sms ? tiles : num_sms);
     return launch_k(kern, dim3(grid), dim3(kThreads), smem, s, pdl, 1, mw, sv, si, sn, P);
   }
 }
@@ -755,16 +992,23 @@ bool down_uses_wide() {
   return env == 1;
 }
 
-cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, bool pdl,
-                              cudaStream_t s) {
+cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, int32_t *split_ctr,
+                              bool pdl, cudaStream_t s) {
   const int rows = down_uses_pair(v) ? 2 * kBlockM : kBlockM;
   const int blocks = (v.M + rows - 1) / rows;
   if (blocks == 0) return cudaSuccess;
-  return launch_k(k_block_path, dim3(blocks), dim3(256), 0, s, pdl, 1, v, crossover, rows, blk_path);
+  return launch_k(k_block_path, dim3(blocks), dim3(256), 0, s, pdl, 1, v, crossover, rows, blk_path,
+                  split_ctr);
+}
+
+size_t split_ws_bytes(int M, int d_model) {
+  if (decode_down_eligible(M) || d_model <= kBN) return 0;
+  return 1024 + 2 * static_cast<size_t>(kMaxSplitCtas) * kSplitPartBytes;
 }
 
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                            const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s) {
+                            const int32_t *blk_path, const SplitWs &split, int num_sms, bool pdl,
+                            cudaStream_t s) {
   if (v.M == 0) return cudaSuccess;
   CUtensorMap mw;
   if (encode_tensor_map_2d(&mw, w_down, d, v.f, static_cast<uint64_t>(d) * 2, 64, kBlockK,
@@ -779,6 +1023,9 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   P.num_kb = (v.f + kBlockK - 1) / kBlockK;
   P.blk_path = blk_path;
   const int ev = (v.E % 8 == 0 && v.E <= 64) ? v.E / 8 : 0;
+  P.split = 0; P.nc = 1; P.ck = 1; P.units = 0; P.grid = 0;
+  P.tiles = 0; P.parts = 1; P.dp_tiles = 0; P.sk_grid = 0;
+  P.part = split.part; P.split_ctr = split.ctr;
   // Slot records by TMA: the row pitches of vals / idx / nnz must be multiples of
   // 16 bytes and every box start 16-byte aligned (ell_w % 8 == 0, T % 8 == 0).
   const int ib = (v.E % 16 == 0) ? v.E : v.E + 8;
@@ -802,6 +1049,46 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   const int tile_m = pair ? 2 * kBlockM : kBlockM;
   P.num_m_blocks = (v.M + tile_m - 1) / tile_m;
   P.num_n_blocks = (d + (wide ? 2 : 1) * kBN - 1) / ((wide ? 2 : 1) * kBN);
+  // Split schedules (512-column tiles, fast builders), chosen so the CTAs that
+  // share a tile stay few and the ones streaming W_down stay in step:
+  //   fewer tiles than SMs: each tile's K steps cut into `parts` equal ranges
+  //     (parts = SMs / tiles, each range at least kMinSplitSteps K steps);
+  //   otherwise, unless the tiles fill whole waves: every tile's chunks dealt
+  //     out evenly over the SMs.  (Full waves of whole tiles followed by a
+  //     shared last wave measured slower on the 2B gated and heavy-tail layers:
+  //     per-tile costs differ there, and an even deal of all chunks averages
+  //     them out.)
+  if (wide && ev > 0 && split.part != nullptr && split.ctr != nullptr && split_ws_bytes(v.M, d) > 0) {
+    constexpr int kMinSplitSteps = 32;
+    const int g = num_sms < kMaxSplitCtas ? num_sms : kMaxSplitCtas;
+    const int tiles = P.num_m_blocks * P.num_n_blocks;
+    P.ck = v.tw > kBlockK ? v.tw / kBlockK : 1;
+    P.nc = (P.num_kb + P.ck - 1) / P.ck;
+    P.tiles = tiles;
+    if (tiles < g) {
+      int parts = g / tiles;
+      const int by_work = (P.nc * P.ck) / kMinSplitSteps;
+      if (parts > by_work) parts = by_work;
+      if (parts > P.nc) parts = P.nc;
+      if (parts >= 2) {
+        P.split = 1;
+        P.parts = parts;
+        P.grid = tiles * parts;
+      }
+    } else {
+      const int rem = tiles % g;
+      if (rem != 0) {
+        P.dp_tiles = 0;
+        P.units = static_cast<long long>(tiles) * P.nc;
+        long long sk = (P.units * P.ck) / kMinSplitSteps;
+        if (sk > g) sk = g;
+        if (sk < 1) sk = 1;
+        P.split = 2;
+        P.sk_grid = static_cast<int>(sk);
+        P.grid = g;
+      }
+    }
+  }
   const size_t b_stage = pair ? kBBytes / 2 : kBBytes;
   // Pipeline depth from the 227 KB budget.  A deep slot ring (4 hidden tiles)
   // only pays while the pipeline keeps at least 4 stages: at wide ell_w it is

@@ -8,9 +8,6 @@
 
 namespace twell {
 
-cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, bool pdl,
-                              cudaStream_t s);
-
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -75,16 +72,34 @@ struct Ws {
   WsLayout L;
   size_t blk_path;   // [M / 128 + 1] i32: down path of each 128-token block
   size_t l1_part;    // [M][T] fp32: per (token, tile) sums of |h| (statistics)
+  size_t split;      // split schedule of the tensor-core down-projection (last;
+                     // present when d_model is given and the shape can use it)
+  size_t split_bytes;
   size_t total;
 };
 
-Ws ws_plan(int M, int d_ff, int tile_w, int cap) {
+// d_model = 0: the regions of the calls that never run the down-projection.
+Ws ws_plan(int M, int d_ff, int tile_w, int cap, int d_model = 0) {
   Ws w;
   w.L = ws_layout(M, tile_w, cap);
   w.blk_path = w.L.total;
   w.l1_part = align256(w.blk_path + sizeof(int32_t) * static_cast<size_t>((M + kBlockM - 1) / kBlockM + 1));
-  w.total = align256(w.l1_part + sizeof(float) * static_cast<size_t>(M) * (d_ff / tile_w));
+  w.split = align256(w.l1_part + sizeof(float) * static_cast<size_t>(M) * (d_ff / tile_w));
+  w.split_bytes = d_model > 0 ? split_ws_bytes(M, d_model) : 0;
+  w.total = align256(w.split + w.split_bytes);
   return w;
+}
+
+SplitWs split_ptrs(const Ws &w, void *ws) {
+  SplitWs sp;
+  sp.part = nullptr;
+  sp.ctr = nullptr;
+  if (w.split_bytes > 0) {
+    uint8_t *base = static_cast<uint8_t *>(ws) + w.split;
+    sp.ctr = reinterpret_cast<int32_t *>(base);
+    sp.part = reinterpret_cast<float *>(base + 1024);
+  }
+  return sp;
 }
 
 PackTarget make_target(const twell_matrix *a, void *ws) {
@@ -123,8 +138,8 @@ twell_status reset_for_pack(const PackTarget &t, cudaStream_t s) {
   return from_cuda(e);
 }
 
-twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int cap) {
-  const Ws w = ws_plan(M, d_ff, tile_w, cap);
+twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int cap, int d_model = 0) {
+  const Ws w = ws_plan(M, d_ff, tile_w, cap, d_model);
   if (ws == nullptr || !a16(ws) || ws_bytes < w.total) return TWELL_ERR_WORKSPACE;
   return TWELL_OK;
 }
@@ -187,7 +202,7 @@ twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_
   if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y)) return TWELL_ERR_INVALID_ARG;
   if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
     return TWELL_ERR_INVALID_ARG;
-  return check_ws(ws, ws_bytes, a->M, a->d_ff, a->tile_w, a->ovf_capacity);
+  return check_ws(ws, ws_bytes, a->M, a->d_ff, a->tile_w, a->ovf_capacity, d_model);
 }
 
 // pdl_first: the call's first kernel may be a dependent launch (true only when
@@ -204,15 +219,24 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
   // decode-size batches: the split-K tensor-core kernel streams W_down over every SM
   if (decode_down_eligible(a->M))
     return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, pdl_first, s));
-  if (mode == TWELL_DOWN_MMA)
-    return from_cuda(launch_spmm_mma(v, W_down, d_model, y, nullptr, sms, pdl_first, s));
-  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity);
+  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity, d_model);
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
-  cudaError_t e = launch_block_path(v, kDownCrossoverDensity, blk, pdl_first, s);
-  if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  e = launch_spmm_gather(v, W_down, d_model, y, blk, true, s);
-  if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sms, true, s));
+  const SplitWs sp = split_ptrs(w, ws);
+  // The block pass also zeroes the split schedule's counters.  MMA mode hands
+  // the tensor-core kernel no block flags: its W_down stream starts before the
+  // kernel waits for its predecessor, and with no gather launch in between that
+  // predecessor is the block pass itself.
+  const bool mma_only = mode == TWELL_DOWN_MMA;
+  if (!mma_only || sp.ctr != nullptr) {
+    cudaError_t e = launch_block_path(v, mma_only ? -1.0f : kDownCrossoverDensity, blk, sp.ctr, pdl_first, s);
+    if (e != cudaSuccess) return TWELL_ERR_CUDA;
+    pdl_first = true;
+  }
+  if (!mma_only) {
+    cudaError_t e = launch_spmm_gather(v, W_down, d_model, y, blk, true, s);
+    if (e != cudaSuccess) return TWELL_ERR_CUDA;
+  }
+  return from_cuda(launch_spmm_mma(v, W_down, d_model, y, mma_only ? nullptr : blk, sp, sms, pdl_first, s));
 }
 
 // Workspace of twell_ffn_backward (every region 256-byte aligned).
@@ -223,7 +247,7 @@ struct BwLayout {
   WsLayout stage_L;
 };
 
-BwLayout bw_layout(int M, int d_ff, int tile_w, int ell_w, int cap, int ell_t, int cap_t) {
+BwLayout bw_layout(int M, int d_model, int d_ff, int tile_w, int ell_w, int cap, int ell_t, int cap_t) {
   BwLayout b;
   const size_t T = d_ff / tile_w, Tt = M / 128, F = d_ff;
   size_t o = 0;
@@ -241,7 +265,7 @@ BwLayout bw_layout(int M, int d_ff, int tile_w, int ell_w, int cap, int ell_t, i
   b.db_part = take(4 * F * Tt);
   b.stage_L = ws_layout(d_ff, 128, cap_t);
   b.stage = take(b.stage_L.total);
-  const size_t s1 = ws_plan(M, d_ff, tile_w, cap).total, s2 = ws_plan(d_ff, M, 128, cap_t).total;
+  const size_t s1 = ws_plan(M, d_ff, tile_w, cap, d_model).total, s2 = ws_plan(d_ff, M, 128, cap_t, d_model).total;
   b.spmm = take(s1 > s2 ? s1 : s2);
   b.total = o;
   return b;
@@ -266,7 +290,7 @@ TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int cap_tok) {
   L.d_nnz = take(2 * static_cast<size_t>(cap_tok) * T);
   L.y_dense = take(2 * static_cast<size_t>(cap_tok) * d_model);
   L.words = take(64);
-  const size_t s1 = ws_plan(M, d_ff, tile_w, 0).total, s2 = ws_plan(cap_tok, d_ff, tile_w, 0).total;
+  const size_t s1 = ws_plan(M, d_ff, tile_w, 0, d_model).total, s2 = ws_plan(cap_tok, d_ff, tile_w, 0, d_model).total;
   L.spmm = take(s1 > s2 ? s1 : s2);
   L.total = o;
   return L;
@@ -313,7 +337,7 @@ size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w
                              int ovf_capacity) {
   if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0) return 0;
   if (d_model <= 0 || d_model % 64 != 0 || (gated != 0 && gated != 1)) return 0;
-  return ws_plan(M, d_ff, tile_w, ovf_capacity).total;
+  return ws_plan(M, d_ff, tile_w, ovf_capacity, d_model).total;
 }
 
 twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
@@ -387,7 +411,7 @@ size_t twell_backward_workspace_bytes(int M, int d_model, int d_ff, int tile_w, 
   if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0 || ovf_capacity_t < 0) return 0;
   if (d_model <= 0 || d_model % 64 != 0 || M % 128 != 0 || d_ff % 128 != 0 || tile_w > 128) return 0;
   if (ell_w_t < 1 || ell_w_t > 128) return 0;
-  return bw_layout(M, d_ff, tile_w, ell_w, ovf_capacity, ell_w_t, ovf_capacity_t).total;
+  return bw_layout(M, d_model, d_ff, tile_w, ell_w, ovf_capacity, ell_w_t, ovf_capacity_t).total;
 }
 
 twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const uint16_t *W_down,
@@ -407,7 +431,7 @@ twell_status twell_ffn_backward(const uint16_t *x, const uint16_t *W_up, const u
   const void *ptrs[] = {x, W_up, W_down, dY, dX, dW_up, db, dW_down};
   for (const void *q : ptrs)
     if (q == nullptr || !a16(q)) return TWELL_ERR_INVALID_ARG;
-  const BwLayout L = bw_layout(M, f, tw, E, h->ovf_capacity, ell_w_t, ovf_capacity_t);
+  const BwLayout L = bw_layout(M, d_model, f, tw, E, h->ovf_capacity, ell_w_t, ovf_capacity_t);
   if (ws == nullptr || !a16(ws) || ws_bytes < L.total) return TWELL_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int sms = sm_count();

@@ -125,12 +125,35 @@ struct UpArgs {
 };
 cudaError_t launch_up_pack(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
 
+// Split schedule of the tensor-core down-projection (128-token x 512-column
+// tiles): the tiles' K steps, in hidden-tile chunks, are dealt out evenly over
+// up to kMaxSplitCtas persistent CTAs, so every SM gets the same share however
+// the tile count falls against the SM count.  A tile shared by several CTAs is
+// summed from their fp32 partial tiles, in CTA order, by the last one to finish.
+// Workspace: one arrival counter per CTA (zeroed by launch_block_path before
+// every launch) and two partial tiles per CTA.
+constexpr int kMaxSplitCtas = 160;
+constexpr size_t kSplitPartBytes = static_cast<size_t>(kBlockM) * 512 * 4;
+struct SplitWs {
+  float *part;     // [2 * kMaxSplitCtas][kSplitPartBytes / 4], or NULL: no split
+  int32_t *ctr;    // [kMaxSplitCtas]
+};
+// Workspace bytes of the split schedule for M tokens and d_model columns
+// (0 when that shape never takes the split kernel).
+size_t split_ws_bytes(int M, int d_model);
+
 // blk_path: NULL (the kernel owns every token block) or one int per 128-token
 // block: 0 = gather path owns it, 1 = tensor-core path owns it.
 cudaError_t launch_spmm_gather(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
                                const int32_t *blk_path, bool pdl, cudaStream_t s);
 cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                            const int32_t *blk_path, int num_sms, bool pdl, cudaStream_t s);
+                            const int32_t *blk_path, const SplitWs &split, int num_sms, bool pdl,
+                            cudaStream_t s);
+// Per 128-token block (256 with CTA pairs): the down path by density against
+// `crossover` (a negative crossover sends every block to the tensor cores); also
+// zeroes the split schedule's arrival counters (split_ctr may be NULL).
+cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, int32_t *split_ctr,
+                              bool pdl, cudaStream_t s);
 
 // Exclusive scan of t.row_ovf into t.row_prefix; the total goes to *t.n_ovf
 // (TWELL_ERR_OVERFLOW_CAPACITY in t.status when above t.cap).

@@ -312,7 +312,7 @@ def run_ours(args):
                            "useful_flop": rl["useful_flop"],
                            "unavoidable_bytes": rl["unavoidable_bytes"],
                            "touched_w_down_rows": touched, "peaks": peaks["source"]},
-        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down),
+        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d),
         "wall_s_timed_region": wall,
     }
     result["clocks"] = clk.summary()
@@ -363,13 +363,19 @@ def _decode_paths(M, f, tw, mode):
     return (M <= 256 and tw <= 128 and f % 128 == 0), (M <= 256 and mode != "gather")
 
 
-def _kernels_per_step(mode, dec_down=False):
+def _kernels_per_step(mode, dec_down=False, d_model=0):
     # up_pack: the producer + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds
     # k_block_path and launches both down kernels (each skips the token blocks
-    # the other owns); the decode-size down path is one kernel
+    # the other owns); mma runs k_block_path too when the split schedule is
+    # possible (d_model > 256: it zeroes the arrival counters); the decode-size
+    # down path is one kernel
     if dec_down:
         return 3 + 1
-    return 3 + (3 if mode == "auto" else 1)
+    if mode == "auto":
+        return 3 + 3
+    if mode == "mma":
+        return 3 + (2 if d_model > 256 else 1)
+    return 3 + 1
 
 
 def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):
