@@ -524,16 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int other = sh.cta(0) == me ? sh.cta(1) : sh.cta(0);
             const float4 *src = part + static_cast<size_t>(sh.slot(other)) * kPartF4 + row_in_tile;
             float4 qa[8], qb[8];
-            auto add_store = [&](const uint32_t (&v)[32], const float4 (&q)[8], int c) {
-              uint32_t w[32];
+            auto add_store = [&](uint32_t (&v)[32], const float4 (&q)[8], int c) {
 #pragma unroll
               for (int j = 0; j < 8; ++j) {
-                w[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + q[j].x);
-                w[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + q[j].y);
-                w[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q[j].z);
-                w[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q[j].w);
+                v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) + q[j].x);
+                v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) + q[j].y);
+                v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) + q[j].z);
+                v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) + q[j].w);
               }
-              store_y(w, c);
+              store_y(v, c);
             };
 #pragma unroll
             for (int j = 0; j < 8; ++j) qa[j] = __ldcs(src + j * kBlockM);

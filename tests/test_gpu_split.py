@@ -85,10 +85,11 @@ def test_split_spmm_against_oracle(M, d, f, tw, E, rho, mode):
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
 
 
-def test_split_mixed_paths_auto():
+@pytest.mark.parametrize("M,d,f", [(896, 1024, 4096), (4864, 2048, 3072)])
+def test_split_mixed_paths_auto(M, d, f):
     """AUTO with some 128-token blocks below the gather crossover: the split
-    schedule skips the gather-owned tiles and the shared ones still add up."""
-    M, d, f, tw, E = 896, 1024, 4096, 128, 16
+    schedules skip the gather-owned tiles and the shared ones still add up."""
+    tw, E = 128, 16
     assert _shared_tiles(M, d, f, tw)
     L = S.small_random(M, d, f, tw, E, 0.05, seed=11)
     h = O.hidden(L.x, L.w_up, L.b)
@@ -148,3 +149,23 @@ def test_split_forward_replays_from_a_cuda_graph():
     ref, y64 = O.ffn_forward(L2.x, L.w_up, L.b, L.w_down, tw, E)
     assert_y_close(y_graph, y64)
     del g
+
+
+def test_split_backward_dx():
+    """The backward's dX = dZ W_up runs through the same down kernels: at this
+    shape its 8 tiles are split two ways (64 K steps each)."""
+    M, d, f, tw, E = 512, 1024, 4096, 128, 16
+    assert _shared_tiles(M, d, f, tw)
+    L = S.small_random(M, d, f, tw, E, 0.05, seed=21)
+    rng = np.random.default_rng(5)
+    dy = S.bf16_bits_from_f32(rng.standard_normal((M, d)).astype(np.float32))
+    x, wu, b, wd = dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_down)
+    y, h = T.twell_ffn_forward(x, wu, b, wd, tile_w=tw, ell_w=E, ovf_capacity=M * (f // tw))
+    assert T.read_status(h)[0] == 0
+    dX, dWu, db, dWd = T.twell_ffn_backward(x, wu, wd, h, dev(dy))
+    assert T.read_status(h)[0] == 0
+    got, _ = twell_to_np(h)
+    g = O.ffn_backward(L.x, L.w_up, L.b, L.w_down, dy, h=O.twell_unpack(got))
+    for name, t in (("dx", dX), ("dw_up", dWu), ("dw_down", dWd)):
+        gg = t.float().cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(gg - g[name]) <= 2e-3 * np.linalg.norm(g[name]), name
