@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
                   const __grid_constant__ CUtensorMap tmap_g, const DecUpParams P) {
   constexpr int WPT = TW / 32;                            // epilogue warps per hidden tile
   constexpr int W_BYTES = (GATED ? 2 : 1) * kWBytes;     // [W_up tile][W_gate tile]
+  griddep_launch_dependents();   // the backup scan waits for this grid anyway
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);

@@ -17,6 +17,7 @@ namespace {
 template <int TW>
 __global__ void __launch_bounds__(256) k_pack_dense(const uint16_t *__restrict__ h, int ld_h,
                                                     PackTarget p) {
+  griddep_launch_dependents();   // the backup scan waits for this grid anyway
   constexpr int EPL = TW / 32;  // elements per lane (1, 2, 4, 8)
   const int lane = threadIdx.x & 31;
   const int warps_per_cta = blockDim.x >> 5;
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
   __shared__ int warp_sums[32];
   __shared__ int carry_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  griddep_launch_dependents();
   griddep_wait();   // the producer's counts
   int carry = 0;
   for (int base = 0; base < p.M; base += 1024 * 8) {
@@ -154,6 +156,7 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
 // Move each staged segment to its rank in the ascending r*T+t order.
 template <int TW>
 __global__ void __launch_bounds__(256) k_ovf_scatter(PackTarget p) {
+  griddep_launch_dependents();
   griddep_wait();   // the row prefix
   const int lane = threadIdx.x & 31;
   const int warps_per_cta = blockDim.x >> 5;

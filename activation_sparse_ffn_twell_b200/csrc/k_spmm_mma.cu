@@ -873,6 +873,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // for each 128-token block of the group so both down kernels read one array.
 __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover, int rows,
                                                     int32_t *blk_path, int32_t *split_ctr) {
+  // The next kernel (gather, or the tensor-core kernel with no block flags)
+  // reads nothing of this one before its own wait.
+  griddep_launch_dependents();
   griddep_wait();   // the counts of the TwELL producer
   // the split schedule's arrival counters start every launch at zero
   if (split_ctr != nullptr && blockIdx.x == 0 && threadIdx.x < kMaxSplitCtas) split_ctr[threadIdx.x] = 0;

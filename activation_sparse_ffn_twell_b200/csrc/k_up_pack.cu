@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const __grid_constant__ CUtensorMap tmap_g, const UpParams P) {
   using C = UpCfg<TW, GATED, PAIR>;
   constexpr int kStages = C::STAGES;
+  griddep_launch_dependents();   // the backup scan waits for this grid anyway
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);

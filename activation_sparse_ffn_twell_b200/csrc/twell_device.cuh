@@ -41,6 +41,12 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_fl
 // Wait until the grids this one depends on (programmatic dependent launch) have
 // completed and their writes are visible; a no-op when launched without it.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel of a dependent launch be scheduled now.  Its blocks run
+// only the work that reads nothing this kernel writes until their
+// griddep_wait(), which still waits for this whole grid to finish.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // Record an asynchronous error in the caller's status word (first error wins).
 __device__ __forceinline__ void raise_status(int32_t *status, int32_t code) {
