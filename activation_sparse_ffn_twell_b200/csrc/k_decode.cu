@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue + pack
+    griddep_wait();   // the call's reset kernel (counters, status) precedes the writes
     // thread = hidden unit (TMEM lane); a hidden tile spans WPT warps, whose
     // nonzero counts are combined through shared memory per 32-token chunk.
     // kDecEpiGroups groups of 4 warps (one per TMEM lane quarter) take the
@@ -685,8 +686,8 @@ cudaError_t launch_up_dec_impl(const UpArgs &a, const PackTarget &t, int num_sms
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = P.num_ub < num_sms ? P.num_ub : num_sms;
-  k_up_pack_dec<TW, GATED><<<grid, kDecUpThreads, smem, s>>>(mx, mw, mg, P);
-  return cudaGetLastError();
+  // a dependent launch after the call's reset kernel (see the epilogue's wait)
+  return launch_k(k_up_pack_dec<TW, GATED>, dim3(grid), dim3(kDecUpThreads), smem, s, true, 1, mx, mw, mg, P);
 }
 
 // Largest number of co-resident clusters of `split` CTAs of the down kernel

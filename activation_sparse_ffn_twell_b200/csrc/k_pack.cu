@@ -18,6 +18,7 @@ template <int TW>
 __global__ void __launch_bounds__(256) k_pack_dense(const uint16_t *__restrict__ h, int ld_h,
                                                     PackTarget p) {
   griddep_launch_dependents();   // the backup scan waits for this grid anyway
+  griddep_wait();                // the call's reset kernel
   constexpr int EPL = TW / 32;  // elements per lane (1, 2, 4, 8)
   const int lane = threadIdx.x & 31;
   const int warps_per_cta = blockDim.x >> 5;
@@ -224,13 +225,29 @@ cudaError_t launch_pack_dense(const uint16_t *h, int ld_h, const PackTarget &t, 
   if (pairs == 0) return cudaSuccess;
   const int grid = grid_for(pairs, 8, 148 * 64);
   switch (t.tw) {
-    case 32: k_pack_dense<32><<<grid, 256, 0, s>>>(h, ld_h, t); break;
-    case 64: k_pack_dense<64><<<grid, 256, 0, s>>>(h, ld_h, t); break;
-    case 128: k_pack_dense<128><<<grid, 256, 0, s>>>(h, ld_h, t); break;
-    case 256: k_pack_dense<256><<<grid, 256, 0, s>>>(h, ld_h, t); break;
+    case 32: return launch_k(k_pack_dense<32>, dim3(grid), dim3(256), 0, s, true, 1, h, ld_h, t);
+    case 64: return launch_k(k_pack_dense<64>, dim3(grid), dim3(256), 0, s, true, 1, h, ld_h, t);
+    case 128: return launch_k(k_pack_dense<128>, dim3(grid), dim3(256), 0, s, true, 1, h, ld_h, t);
+    case 256: return launch_k(k_pack_dense<256>, dim3(grid), dim3(256), 0, s, true, 1, h, ld_h, t);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+}
+
+// The status word and the staging counters of a producer call start at zero.
+// The producer that follows is a dependent launch: its loads and MMAs overlap
+// this kernel, its writes wait for it.
+__global__ void __launch_bounds__(256) k_pack_reset(int32_t *status, int32_t *words, int n) {
+  griddep_launch_dependents();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i == 0) *status = 0;
+  for (int k = i; k < n; k += gridDim.x * blockDim.x) words[k] = 0;
+}
+
+cudaError_t launch_pack_reset(const PackTarget &t, cudaStream_t s) {
+  // [stage_ctr, row_ovf + M): the counter, the per-token counts and the padding between
+  const int n = static_cast<int>((t.row_ovf + t.M) - t.stage_ctr);
+  const int grid = n / 256 + 1 < 148 ? n / 256 + 1 : 148;
+  return launch_k(k_pack_reset, dim3(grid), dim3(256), 0, s, false, 1, t.status, t.stage_ctr, n);
 }
 
 cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {

@@ -221,6 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // The loads and MMAs above read only x and the weights; the epilogue writes
+    // the packed output, the staging counters and the status word, which the
+    // call's reset kernel zeroes first.
+    griddep_wait();
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const int row_in_tile = q * 32 + lane;
     uint32_t *my_slots = sSlotw + row_in_tile * pitch_w;
@@ -456,12 +460,12 @@ cudaError_t launch_up_impl(const UpArgs &a, const PackTarget &t, int num_sms, cu
     }
     int pairs = max_pairs < num_sms / 2 ? max_pairs : num_sms / 2;
     if (pairs > tiles) pairs = tiles;
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    return cudaLaunchKernelEx(&cfg, k_up_pack<TW, GATED, true>, mx, mw, mg, P);
+    // a dependent launch after the call's reset kernel (see the epilogue's wait)
+    return launch_k(k_up_pack<TW, GATED, true>, dim3(2 * pairs), dim3(kThreads), smem, s, true, 2, mx, mw,
+                    mg, P);
   } else {
     const int grid = tiles < num_sms ? tiles : num_sms;
-    k_up_pack<TW, GATED, false><<<grid, kThreads, smem, s>>>(mx, mw, mg, P);
-    return cudaGetLastError();
+    return launch_k(k_up_pack<TW, GATED, false>, dim3(grid), dim3(kThreads), smem, s, true, 1, mx, mw, mg, P);
   }
 }
 

@@ -129,13 +129,10 @@ TwellView make_view(const twell_matrix *a) {
 
 twell_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TWELL_OK : TWELL_ERR_CUDA; }
 
-// Reset the status word and the overflow staging counters before a producer runs.
+// Reset the status word and the overflow staging counters before a producer
+// runs (one kernel; the producer overlaps it as a dependent launch).
 twell_status reset_for_pack(const PackTarget &t, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(t.status, 0, sizeof(int32_t), s);
-  if (e != cudaSuccess) return TWELL_ERR_CUDA;
-  const size_t bytes = reinterpret_cast<uint8_t *>(t.row_ovf + t.M) - reinterpret_cast<uint8_t *>(t.stage_ctr);
-  e = cudaMemsetAsync(t.stage_ctr, 0, bytes, s);
-  return from_cuda(e);
+  return from_cuda(launch_pack_reset(t, s));
 }
 
 twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int cap, int d_model = 0) {

@@ -155,6 +155,11 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
 cudaError_t launch_block_path(const TwellView &v, float crossover, int32_t *blk_path, int32_t *split_ctr,
                               bool pdl, cudaStream_t s);
 
+// Zero the status word and the staging counters before a producer; the
+// producers (launch_up_pack, launch_up_pack_decode, launch_pack_dense) are
+// dependent launches that must directly follow it.
+cudaError_t launch_pack_reset(const PackTarget &t, cudaStream_t s);
+
 // Exclusive scan of t.row_ovf into t.row_prefix; the total goes to *t.n_ovf
 // (TWELL_ERR_OVERFLOW_CAPACITY in t.status when above t.cap).
 cudaError_t launch_row_scan(const PackTarget &t, bool pdl, cudaStream_t s);

@@ -96,8 +96,7 @@ extern "C" twell_status twell_pack_noalloc(const uint16_t *h, int M, int d_ff, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // The array keeps whatever the previous call left in it: the status word, the
   // staging counter and the per-token overflow counts must start at zero.
-  if (cudaMemsetAsync(t.status, 0, sizeof(int32_t), s) != cudaSuccess) return TWELL_ERR_CUDA;
-  if (cudaMemsetAsync(base + L.ctr, 0, L.row_prefix - L.ctr, s) != cudaSuccess) return TWELL_ERR_CUDA;
+  if (launch_pack_reset(t, s) != cudaSuccess) return TWELL_ERR_CUDA;
   if (launch_pack_dense(h, ld_h, t, s) != cudaSuccess) return TWELL_ERR_CUDA;
   return launch_overflow_finalize(t, s) == cudaSuccess ? TWELL_OK : TWELL_ERR_CUDA;
 }

@@ -364,18 +364,18 @@ def _decode_paths(M, f, tw, mode):
 
 
 def _kernels_per_step(mode, dec_down=False, d_model=0):
-    # up_pack: the producer + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds
+    # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds
     # k_block_path and launches both down kernels (each skips the token blocks
     # the other owns); mma runs k_block_path too when the split schedule is
     # possible (d_model > 256: it zeroes the arrival counters); the decode-size
     # down path is one kernel
     if dec_down:
-        return 3 + 1
+        return 4 + 1
     if mode == "auto":
-        return 3 + 3
+        return 4 + 3
     if mode == "mma":
-        return 3 + (2 if d_model > 256 else 1)
-    return 3 + 1
+        return 4 + (2 if d_model > 256 else 1)
+    return 4 + 1
 
 
 def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):

@@ -3,7 +3,7 @@
 * The bounded shared-memory-barrier wait used by every tensor-core kernel gives
   up by itself on a barrier nothing arrives on, reports TWELL_ERR_TIMEOUT, and
   leaves the context usable (no fault, no hang: the wait has a wall-clock limit).
-* The whole forward (memsets, producer, backup ordering, down kernels, chained
+* The whole forward (reset kernel, producer, backup ordering, down kernels, chained
   as dependent launches) captures into a CUDA graph and replays to the same
   bits as eager calls, for both the token-major and the decode-size kernels.
 """
