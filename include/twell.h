@@ -90,7 +90,10 @@ const char *twell_status_string(twell_status s);
 /*
  * Workspace bytes needed by twell_pack / twell_up_pack / twell_spmm /
  * twell_ffn_forward for these sizes (the maximum over the four calls).  gated is
- * 0 or 1.  Returns 0 for invalid shapes.
+ * 0 or 1.  Returns 0 for invalid shapes.  The workspace is scratch: its contents
+ * need no initialisation and are undefined after a call.  For M > 256 and
+ * d_model > 256 it includes 80 MiB of fp32 partial tiles used when the
+ * tensor-core down-projection shares 128 x 512 tiles of y between SMs.
  */
 size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w, int gated,
                              int ovf_capacity);
