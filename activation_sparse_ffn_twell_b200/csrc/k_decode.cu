@@ -40,6 +40,10 @@ constexpr int kDecEpiGroups = 3;                         // up epilogue: groups 
 constexpr int kDecUpThreads = 64 + kDecEpiGroups * 128;   // TMA, MMA, epilogue warps
 constexpr int kDecDownThreads = 448;                     // TMA, MMA, 4 epilogue, 8 builder warps
 constexpr size_t kDecSmemBudget = 225 * 1024;
+// K steps per pipeline stage of the up kernel: two adjacent 64-column boxes of
+// each weight row per stage, so the rows are read in 256-byte pieces (one K step
+// per stage when gated: W_up and W_gate tiles already fill a stage).
+template <bool GATED> constexpr int dec_up_kps() { return GATED ? 1 : 2; }
 
 uint32_t tmem_cols_for(int cols) {
   uint32_t c = 32;
@@ -71,7 +75,9 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const int kStages = P.stages;
-  const int STAGE = W_BYTES + P.np * 128;                 // [W_up tile][W_gate tile][x tile]
+  constexpr int KPS = dec_up_kps<GATED>();
+  const int XB = P.np * 128;                              // x tile of one K step
+  const int STAGE = KPS * (W_BYTES + XB);                 // [KPS weight tiles][KPS x tiles]
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * STAGE);
   uint64_t *full = bars;
   uint64_t *empty = bars + kDecMaxStages;
@@ -112,16 +118,21 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
       uint32_t filled = 0;
       bool ok = true;
       for (int ub = blockIdx.x; ub < P.num_ub && ok; ub += gridDim.x) {
-        for (int kb = 0; kb < P.num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < P.num_kb; kb0 += KPS) {
+          const int nk = min(KPS, P.num_kb - kb0);
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           // the x box is M rows; operand rows M..np-1 feed accumulator columns
           // that no one reads
-          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(W_BYTES + P.M * 128));
+          mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nk * (W_BYTES + P.M * 128)));
           filled |= 1u << stage;
           uint8_t *dst = smem + stage * STAGE;
-          tma_load_2d(dst, &tmap_w, &full[stage], kb * kBlockK, ub * kDecUnits);
-          if constexpr (GATED) tma_load_2d(dst + kWBytes, &tmap_g, &full[stage], kb * kBlockK, ub * kDecUnits);
-          tma_load_2d(dst + W_BYTES, &tmap_x, &full[stage], kb * kBlockK, 0);
+          for (int j = 0; j < nk; ++j) {
+            const int kb = kb0 + j;
+            tma_load_2d(dst + j * W_BYTES, &tmap_w, &full[stage], kb * kBlockK, ub * kDecUnits);
+            if constexpr (GATED)
+              tma_load_2d(dst + j * W_BYTES + kWBytes, &tmap_g, &full[stage], kb * kBlockK, ub * kDecUnits);
+            tma_load_2d(dst + KPS * W_BYTES + j * XB, &tmap_x, &full[stage], kb * kBlockK, 0);
+          }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
@@ -143,20 +154,24 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
       for (int ub = blockIdx.x; ub < P.num_ub && ok; ub += gridDim.x, ++it) {
         if (!mbar_wait(tm_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        for (int kb = 0; kb < P.num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < P.num_kb; kb0 += KPS) {
+          const int nk = min(KPS, P.num_kb - kb0);
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t w_addr = smem_u32(smem + stage * STAGE);
-          const uint32_t x_addr = w_addr + W_BYTES;
+          const uint32_t s_addr = smem_u32(smem + stage * STAGE);
+          for (int j = 0; j < nk; ++j) {
+            const uint32_t w_addr = s_addr + j * W_BYTES;
+            const uint32_t x_addr = s_addr + KPS * W_BYTES + j * XB;
 #pragma unroll
-          for (int k = 0; k < kBlockK / kUmmaK; ++k) {
-            const uint64_t xdesc = smem_desc_sw128(x_addr + k * 32, 16, 1024);
-            const uint32_t acc = (kb | k) != 0;
-            if constexpr (GATED) {
-              umma_bf16(tmem_base, smem_desc_sw128(w_addr + kWBytes + k * 32, 16, 1024), xdesc, P.idesc, acc);
-              umma_bf16(tmem_base + P.acc_up, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
-            } else {
-              umma_bf16(tmem_base, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
+            for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+              const uint64_t xdesc = smem_desc_sw128(x_addr + k * 32, 16, 1024);
+              const uint32_t acc = ((kb0 + j) | k) != 0;
+              if constexpr (GATED) {
+                umma_bf16(tmem_base, smem_desc_sw128(w_addr + kWBytes + k * 32, 16, 1024), xdesc, P.idesc, acc);
+                umma_bf16(tmem_base + P.acc_up, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
+              } else {
+                umma_bf16(tmem_base, smem_desc_sw128(w_addr + k * 32, 16, 1024), xdesc, P.idesc, acc);
+              }
             }
           }
           umma_commit(&empty[stage]);
@@ -663,7 +678,8 @@ cudaError_t launch_up_dec_impl(const UpArgs &a, const PackTarget &t, int num_sms
   P.z_debug = a.z_debug;
   P.l1_part = a.l1_part;
   P.out = t;
-  const size_t stage = (GATED ? 2 : 1) * static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
+  const size_t stage = static_cast<size_t>(dec_up_kps<GATED>()) *
+                       ((GATED ? 2 : 1) * static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128);
   const size_t extra = 1024 + 6144;                      // alignment slack, barriers, counts
   int stages = static_cast<int>((kDecSmemBudget - extra) / stage);
   if (stages > kDecMaxStages) stages = kDecMaxStages;
