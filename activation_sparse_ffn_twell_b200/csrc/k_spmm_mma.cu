@@ -8,15 +8,17 @@
 // the dense backup segment of overflowing pairs) -- the dense h never exists in
 // HBM -- and multiplied by the matching 64 rows of W_down.
 //
-// Roles (one CTA per SM, persistent over 128-token x 256- or 512-column tiles
-// of y):
+// Roles (one CTA per SM, persistent over segments: whole 128-token x 256- or
+// 512-column tiles of y, or, on the split schedules, K-step ranges of 512-column
+// tiles whose fp32 partials are summed by the last CTA to finish):
 //   warp 0      TMA: W_down[k0:k0+64, n0:n0+256] as four 64x64 boxes, 128-byte
 //               swizzle; this is an N-major ("MN-major") B operand.  512-column
 //               tiles load two such stages per K step from their own ring.
 //   warp 1      TMEM allocation (512 fp32 columns: two 256-column accumulators,
 //               double-buffered, or both halves of one 512-column tile) +
 //               tcgen05.mma issue.
-//   warps 2..5  epilogue: TMEM -> fp32 registers -> bf16 -> y.
+//   warps 2..5  epilogue: TMEM -> fp32 registers -> bf16 -> y (or -> an fp32
+//               partial tile, counted at the tile's arrival counter).
 //   warps 6..13 A builders.  Fast path (ell_w % 8 == 0): two threads per token
 //               row, each taking alternate slots.  The row's slot record of the
 //               next hidden tile is in registers (or a TMA-fed shared-memory
