@@ -25,7 +25,7 @@ __all__ = [
     "TwellError", "TwELL", "lib", "library_path", "workspace_bytes",
     "twell_pack", "twell_up_pack", "twell_up_pack_stats", "twell_spmm", "twell_ffn_forward",
     "twell_ffn_backward", "twell_spmm_token_overflow", "read_status",
-    "DOWN_MODES", "STATUS", "default_ovf_capacity",
+    "DOWN_MODES", "STATUS", "default_ovf_capacity", "down_schedule",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,7 @@ _SIGS = {
     "twell_read_status": (_I, [ctypes.POINTER(_Matrix), _P, ctypes.POINTER(ctypes.c_int32)]),
     "twell_pack_noalloc": (_I, [_P, _I, _I, _I, _I, _I, ctypes.POINTER(_Matrix), _P]),
     "twell_selftest_bounded_wait": (_I, [_P, _P, _P]),
+    "twell_down_schedule": (_I, [_I, _I, _I, _I, _I, _I, _P, _I]),
     "twell_backward_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "twell_token_overflow_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "twell_spmm_token_overflow": (_I, [ctypes.POINTER(_Matrix), _P, _I, _P, _I, _P, _P,
@@ -358,3 +359,21 @@ def read_status(a: TwELL, stream=None):
     m = a.cstruct()
     code = _lib().twell_read_status(ctypes.byref(m), _stream_handle(stream), ctypes.byref(n))
     return int(code), int(n.value)
+
+
+def down_schedule(M: int, d_model: int, d_ff: int, tile_w: int, ell_w: int, num_sms: int):
+    """The work split of the token-major tensor-core down-projection for these
+    sizes on num_sms SMs, from the library's own planning code (host only).
+    Returns None for shapes that do not take that kernel, else a dict with
+    `split` (0 whole tiles, 1 split-K, 2 even deal of K chunks), `ctas`, `tiles`,
+    `k_steps` and `segments`: (cta, tile, k0, k1, sharers, counter, slot) tuples."""
+    fn = _lib().twell_down_schedule
+    n = fn(M, d_model, d_ff, tile_w, ell_w, num_sms, None, 0)
+    if n < 0:
+        return None
+    buf = (ctypes.c_int32 * n)()
+    fn(M, d_model, d_ff, tile_w, ell_w, num_sms, ctypes.cast(buf, ctypes.c_void_p), n)
+    v = list(buf)
+    segs = [tuple(v[i:i + 7]) for i in range(4, n, 7)]
+    return {"split": v[0], "ctas": v[1], "tiles": v[2], "k_steps": v[3], "segments": segs}
+

@@ -68,11 +68,11 @@ struct DownParams {
   //     tiles c, c + grid, ...; none in the current choice), then the other
   //     tiles' chunks dealt out evenly, numbered tile-major, over the first
   //     sk_grid CTAs: CTA c owns chunks [c U / sk_grid, (c + 1) U / sk_grid).
-  int split;                 // 0 none, 1 split-K, 2 waves + shared remainder
+  int split;                 // 0 none, 1 split-K, 2 shared chunks
   int nc, ck;                // chunks per tile, K steps per chunk
   int tiles, parts;          // (1)
   int dp_tiles, sk_grid;     // (2)
-  long long units;           // (2) chunks of the shared remainder
+  long long units;           // (2) chunks dealt out
   float *part;               // [2 * kMaxSplitCtas][128 x 512] fp32 partial tiles
   int32_t *split_ctr;        // [kMaxSplitCtas] arrivals per shared tile
   int grid;                  // CTAs launched
@@ -97,11 +97,16 @@ __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
   return P.blk_path == nullptr || P.blk_path[m_blk] != 0;
 }
 
-// Schedule 2's shared remainder: CTA c owns chunks [c U / G, (c + 1) U / G).
-__device__ __forceinline__ long long split_begin(int c, long long U, int G) {
+// The schedule helpers below also compile for the host, where
+// twell_down_schedule lists a launch's segments without a GPU.
+__host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ long long lmin(long long a, long long b) { return a < b ? a : b; }
+
+// Schedule 2: CTA c owns chunks [c U / G, (c + 1) U / G) of the U dealt out.
+__host__ __device__ __forceinline__ long long split_begin(int c, long long U, int G) {
   return static_cast<long long>(c) * U / G;
 }
-__device__ __forceinline__ int split_owner(long long q, long long U, int G) {   // CTA of chunk q
+__host__ __device__ __forceinline__ int split_owner(long long q, long long U, int G) {   // CTA of chunk q
   return static_cast<int>(((q + 1) * G + U - 1) / U - 1);
 }
 
@@ -109,9 +114,9 @@ __device__ __forceinline__ int split_owner(long long q, long long U, int G) {   
 // publishes its fp32 partial in slot(cta) and the arrivals are counted at ctr.
 struct Sharing {
   int n, first, stride, ctr;
-  long long ts, U;     // schedule 2: the tile's first remainder chunk, remainder size
+  long long ts, U;     // schedule 2: the tile's first dealt chunk, chunks dealt out
   int G;
-  __device__ __forceinline__ Sharing(const DownParams &P, int tile) {
+  __host__ __device__ __forceinline__ Sharing(const DownParams &P, int tile) {
     if (P.split == 1) {
       n = P.parts; first = tile; stride = P.tiles; ctr = tile; ts = 0; U = 0; G = 0;
     } else {
@@ -122,10 +127,10 @@ struct Sharing {
       stride = 1; ctr = first;
     }
   }
-  __device__ __forceinline__ int cta(int j) const { return first + j * stride; }
+  __host__ __device__ __forceinline__ int cta(int j) const { return first + j * stride; }
   // schedule 2: a CTA's segment in this tile is its last one when its share
   // began at or before the tile (slot 2c + 1), else its first one (slot 2c)
-  __device__ __forceinline__ int slot(int c) const {
+  __host__ __device__ __forceinline__ int slot(int c) const {
     return G == 0 ? 2 * c : 2 * c + (split_begin(c, U, G) <= ts ? 1 : 0);
   }
 };
@@ -135,7 +140,7 @@ struct Sched {
   int mode, c, G, i;
   long long q, qe;
   int tile, kb0, kb1;
-  __device__ __forceinline__ Sched(const DownParams &P, bool split, int unit0, int n_units) {
+  __host__ __device__ __forceinline__ Sched(const DownParams &P, bool split, int unit0, int n_units) {
     mode = split ? P.split : 0;
     c = unit0; G = n_units; i = 0;
     q = qe = 0;
@@ -145,13 +150,13 @@ struct Sched {
     }
     tile = kb0 = kb1 = 0;
   }
-  __device__ __forceinline__ bool next(const DownParams &P) {
+  __host__ __device__ __forceinline__ bool next(const DownParams &P) {
     if (mode == 1) {
       if (i++ > 0) return false;
       tile = c % P.tiles;
       const int p = c / P.tiles;
       kb0 = (p * P.nc / P.parts) * P.ck;
-      kb1 = min(((p + 1) * P.nc / P.parts) * P.ck, P.num_kb);
+      kb1 = imin(((p + 1) * P.nc / P.parts) * P.ck, P.num_kb);
       return true;
     }
     const int whole_end = mode == 2 ? P.dp_tiles : P.num_m_blocks * P.num_n_blocks;
@@ -165,10 +170,10 @@ struct Sched {
     const int r = static_cast<int>(q / P.nc);
     const long long t0 = static_cast<long long>(r) * P.nc;
     const int c0 = static_cast<int>(q - t0);
-    const int c1 = static_cast<int>(min(qe - t0, static_cast<long long>(P.nc)));
+    const int c1 = static_cast<int>(lmin(qe - t0, static_cast<long long>(P.nc)));
     tile = P.dp_tiles + r;
     kb0 = c0 * P.ck;
-    kb1 = min(c1 * P.ck, P.num_kb);
+    kb1 = imin(c1 * P.ck, P.num_kb);
     q = t0 + c1;
     return true;
   }
@@ -914,6 +919,53 @@ __global__ void __launch_bounds__(256) k_block_path(TwellView A, float crossover
   }
 }
 
+// Split schedule of a 512-column-tile launch (P.num_m_blocks, num_n_blocks,
+// num_kb and A set); leaves P.split = 0 when whole tiles are kept.
+void plan_split(DownParams &P, int M, int d, int num_sms) {
+  const int tw = P.A.tw;
+  // Split schedules (512-column tiles, fast builders), chosen so the CTAs that
+  // share a tile stay few and the ones streaming W_down stay in step:
+  //   fewer tiles than SMs: each tile's K steps cut into `parts` equal ranges
+  //     (parts = SMs / tiles, each range at least kMinSplitSteps K steps);
+  //   otherwise, unless the tiles fill whole waves: every tile's chunks dealt
+  //     out evenly over the SMs.  (Full waves of whole tiles followed by a
+  //     shared last wave measured slower on the 2B gated and heavy-tail layers:
+  //     per-tile costs differ there, and an even deal of all chunks averages
+  //     them out.)
+  if (split_ws_bytes(M, d) > 0) {
+    constexpr int kMinSplitSteps = 32;
+    const int g = num_sms < kMaxSplitCtas ? num_sms : kMaxSplitCtas;
+    const int tiles = P.num_m_blocks * P.num_n_blocks;
+    P.ck = tw > kBlockK ? tw / kBlockK : 1;
+    P.nc = (P.num_kb + P.ck - 1) / P.ck;
+    P.tiles = tiles;
+    if (tiles < g) {
+      int parts = g / tiles;
+      const int by_work = (P.nc * P.ck) / kMinSplitSteps;
+      if (parts > by_work) parts = by_work;
+      if (parts > P.nc) parts = P.nc;
+      if (parts >= 2) {
+        P.split = 1;
+        P.parts = parts;
+        P.grid = tiles * parts;
+      }
+    } else {
+      // only when the deal is shorter than the whole-tile waves on every SM
+      const long long waves = (tiles + num_sms - 1) / num_sms;
+      if (tiles % num_sms != 0 && static_cast<long long>(tiles) < waves * g) {
+        P.dp_tiles = 0;
+        P.units = static_cast<long long>(tiles) * P.nc;
+        long long sk = (P.units * P.ck) / kMinSplitSteps;
+        if (sk > g) sk = g;
+        if (sk < 1) sk = 1;
+        P.split = 2;
+        P.sk_grid = static_cast<int>(sk);
+        P.grid = g;
+      }
+    }
+  }
+}
+
 template <int EV, bool TSLOT, bool PAIR, bool WIDE = false>
 cudaError_t launch_down(const CUtensorMap &mw, const CUtensorMap &sv, const CUtensorMap &si,
                         const CUtensorMap &sn, const DownParams &P, int num_sms, size_t smem,
@@ -1053,46 +1105,7 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   const int tile_m = pair ? 2 * kBlockM : kBlockM;
   P.num_m_blocks = (v.M + tile_m - 1) / tile_m;
   P.num_n_blocks = (d + (wide ? 2 : 1) * kBN - 1) / ((wide ? 2 : 1) * kBN);
-  // Split schedules (512-column tiles, fast builders), chosen so the CTAs that
-  // share a tile stay few and the ones streaming W_down stay in step:
-  //   fewer tiles than SMs: each tile's K steps cut into `parts` equal ranges
-  //     (parts = SMs / tiles, each range at least kMinSplitSteps K steps);
-  //   otherwise, unless the tiles fill whole waves: every tile's chunks dealt
-  //     out evenly over the SMs.  (Full waves of whole tiles followed by a
-  //     shared last wave measured slower on the 2B gated and heavy-tail layers:
-  //     per-tile costs differ there, and an even deal of all chunks averages
-  //     them out.)
-  if (wide && ev > 0 && split.part != nullptr && split.ctr != nullptr && split_ws_bytes(v.M, d) > 0) {
-    constexpr int kMinSplitSteps = 32;
-    const int g = num_sms < kMaxSplitCtas ? num_sms : kMaxSplitCtas;
-    const int tiles = P.num_m_blocks * P.num_n_blocks;
-    P.ck = v.tw > kBlockK ? v.tw / kBlockK : 1;
-    P.nc = (P.num_kb + P.ck - 1) / P.ck;
-    P.tiles = tiles;
-    if (tiles < g) {
-      int parts = g / tiles;
-      const int by_work = (P.nc * P.ck) / kMinSplitSteps;
-      if (parts > by_work) parts = by_work;
-      if (parts > P.nc) parts = P.nc;
-      if (parts >= 2) {
-        P.split = 1;
-        P.parts = parts;
-        P.grid = tiles * parts;
-      }
-    } else {
-      const int rem = tiles % g;
-      if (rem != 0) {
-        P.dp_tiles = 0;
-        P.units = static_cast<long long>(tiles) * P.nc;
-        long long sk = (P.units * P.ck) / kMinSplitSteps;
-        if (sk > g) sk = g;
-        if (sk < 1) sk = 1;
-        P.split = 2;
-        P.sk_grid = static_cast<int>(sk);
-        P.grid = g;
-      }
-    }
-  }
+  if (wide && ev > 0 && split.part != nullptr && split.ctr != nullptr) plan_split(P, v.M, d, num_sms);
   const size_t b_stage = pair ? kBBytes / 2 : kBBytes;
   // Pipeline depth from the 227 KB budget.  A deep slot ring (4 hidden tiles)
   // only pays while the pipeline keeps at least 4 stages: at wide ell_w it is
@@ -1136,3 +1149,47 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
 }
 
 }  // namespace twell
+
+// Diagnostic: the segments of a tensor-core down-projection launch, computed on
+// the host by the same planning and scheduling code the kernel runs.
+extern "C" int twell_down_schedule(int M, int d_model, int d_ff, int tile_w, int ell_w, int num_sms,
+                                   int32_t *out, int out_len) {
+  using namespace twell;
+  const bool tw_ok = tile_w == 32 || tile_w == 64 || tile_w == 128 || tile_w == 256;
+  if (M <= 0 || d_model <= 0 || d_model % 64 != 0 || d_ff <= 0 || !tw_ok || d_ff % tile_w != 0 ||
+      ell_w < 1 || ell_w > tile_w || num_sms <= 0)
+    return -1;
+  if (decode_down_eligible(M)) return -1;   // the decode-size kernel has its own split
+  DownParams P = {};
+  P.A.M = M; P.A.f = d_ff; P.A.tw = tile_w; P.A.E = ell_w; P.A.T = d_ff / tile_w;
+  if (down_uses_pair(P.A)) return -1;       // the pair grid needs an occupancy query
+  const int ev = (ell_w % 8 == 0 && ell_w <= 64) ? ell_w / 8 : 0;
+  const bool wide = d_model > kBN && down_uses_wide();
+  P.num_m_blocks = (M + kBlockM - 1) / kBlockM;
+  P.num_n_blocks = (d_model + (wide ? 2 : 1) * kBN - 1) / ((wide ? 2 : 1) * kBN);
+  P.num_kb = (d_ff + kBlockK - 1) / kBlockK;
+  P.nc = 1; P.ck = 1; P.parts = 1;
+  if (wide && ev > 0) plan_split(P, M, d_model, num_sms);
+  const int tiles = P.num_m_blocks * P.num_n_blocks;
+  const int grid = P.split ? P.grid : (tiles < num_sms ? tiles : num_sms);
+  int n = 0;
+  auto put = [&](int v) {
+    if (out != nullptr && n < out_len) out[n] = v;
+    ++n;
+  };
+  put(P.split); put(grid); put(tiles); put(P.num_kb);
+  for (int c = 0; c < grid; ++c) {
+    Sched sc(P, P.split != 0, c, grid);
+    while (sc.next(P)) {
+      put(c); put(sc.tile); put(sc.kb0); put(sc.kb1);
+      if (sc.kb0 == 0 && sc.kb1 == P.num_kb) {
+        put(1); put(-1); put(-1);
+      } else {
+        const Sharing sh(P, sc.tile);
+        put(sh.n); put(sh.ctr); put(sh.slot(c));
+      }
+    }
+  }
+  return n;
+}
+

@@ -243,6 +243,23 @@ twell_status twell_spmm_token_overflow(const twell_matrix *a, const uint16_t *W_
                                        size_t ws_bytes, void *stream);
 
 /*
+ * twell_down_schedule -- diagnostic, host only (no GPU, nothing launched): the
+ * work split of the token-major tensor-core down-projection (twell_spmm, MMA
+ * path, M > 256) for these sizes on a GPU with num_sms SMs, from the same
+ * planning and scheduling code the kernel runs.  Writes at most out_len int32
+ * to out (host memory, may be NULL) and returns the number needed, or -1 for
+ * shapes that do not take this kernel.  Layout: a header
+ *   [split (0 whole tiles, 1 split-K, 2 even deal of K chunks), CTAs, tiles, K steps]
+ * then, per CTA in order and per segment in its order, 7 values
+ *   [cta, tile, first K step, end K step, CTAs sharing the tile (1: whole tile),
+ *    arrival counter index (-1), partial-tile slot (-1)].
+ * Tiles are 128 tokens x 512 columns of y (256 when d_model <= 256).  The paper
+ * has no counterpart.
+ */
+int twell_down_schedule(int M, int d_model, int d_ff, int tile_w, int ell_w, int num_sms, int32_t *out,
+                        int out_len);
+
+/*
  * twell_selftest_bounded_wait -- diagnostic for the failure path.  Every wait of
  * the tensor-core kernels on a shared-memory barrier is bounded (about 2 s of
  * device wall clock); one that gives up records TWELL_ERR_TIMEOUT and the kernel
