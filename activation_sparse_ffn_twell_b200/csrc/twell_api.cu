@@ -315,7 +315,7 @@ using namespace twell;
 
 extern "C" {
 
-int twell_version(void) { return 100; }
+int twell_version(void) { return 200; }
 
 const char *twell_status_string(twell_status s) {
   switch (s) {
