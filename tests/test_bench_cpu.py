@@ -1,0 +1,53 @@
+"""Host-side parts of bench.py that run without a GPU: the reference arm (the
+oracle timed on the host cores) prints one JSON line with the contract's keys,
+the traffic lookup is tied to the kernels' current sources, and the kernel
+count per step follows the launch sequence of the library."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_reference_arm_prints_the_contract_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "0", "--ref-tokens", "16"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT, check=True).stdout
+    line = json.loads(out.strip().splitlines()[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e", "impl"):
+        assert k in line, k
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "relu_ffn_layer_1.5b"
+
+
+def test_traffic_lookup_follows_the_kernel_source(monkeypatch, tmp_path):
+    src = tmp_path / "activation_sparse_ffn_twell_b200" / "csrc"
+    src.mkdir(parents=True)
+    (src / "k_demo.cu").write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench._kernel_source_hash(os.path.join("activation_sparse_ffn_twell_b200", "csrc", "k_demo.cu"))
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(
+        {"w": {"k_demo": {"source": "k_demo.cu", "source_sha256_16": h, "dram_bytes_per_launch": 123}}}))
+    assert bench._ncu_traffic("k_demo", "w") == 123.0
+    assert bench._ncu_traffic("k_demo", "other") is None
+    (src / "k_demo.cu").write_text("// kernel v2\n")            # the kernel changed: no figure
+    assert bench._ncu_traffic("k_demo", "w") is None
+
+
+def test_kernels_per_step():
+    # reset, producer, backup scan, scatter + block pass, gather, tensor-core kernel
+    assert bench._kernels_per_step("auto", False, 2048) == 7
+    # + block pass (split counters) and the tensor-core kernel
+    assert bench._kernels_per_step("mma", False, 2048) == 6
+    assert bench._kernels_per_step("mma", False, 256) == 5
+    assert bench._kernels_per_step("gather", False, 2048) == 5
+    # decode-size: the split-K down kernel alone
+    assert bench._kernels_per_step("auto", True, 4096) == 5
