@@ -286,6 +286,8 @@ def run_ours(args):
     phases = {"up": phase(*up_k, up_flop, up_bytes, up_s),
               "down": phase(*down_k, down_flop, down_bytes, down_s)}
     phases["down"]["executed_tflops"] = 2.0 * M * d * f / down_s / 1e12
+    # the executed (dense-rate) work against the tensor peak, next to the algorithmic frac
+    phases["down"]["executed_frac_of_tensor_peak"] = phases["down"]["executed_tflops"] / peaks["tc_tflops"]
     dom = max(phases, key=lambda k: phases[k]["ms"])
     P_ = phases[dom]
     result = {
