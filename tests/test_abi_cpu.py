@@ -68,6 +68,13 @@ def test_workspace_bytes_rules(L):
     assert L.twell_workspace_bytes(4096, 2048, 8192, 128, 16, 0, -1) == 0       # capacity
     bigger = L.twell_workspace_bytes(4096, 2048, 8192, 128, 16, 0, 8192)
     assert bigger >= ok + 4096 * (128 * 2 + 4)
+    # the tensor-core down kernel's split schedules (M > 256 tokens, d_model > 256):
+    # 160 arrival counters and 2 x 160 fp32 partial tiles of 128 x 512
+    split = 2 * 160 * 128 * 512 * 4
+    narrow = L.twell_workspace_bytes(4096, 256, 8192, 128, 16, 0, 4096)
+    assert ok - narrow >= split
+    small_m = L.twell_workspace_bytes(256, 2048, 8192, 128, 16, 0, 4096)
+    assert small_m < split                      # decode-size batches use their own kernel
 
 
 def _matrix(M=256, f=1024, tw=128, E=16, cap=64, base=0x10000):
