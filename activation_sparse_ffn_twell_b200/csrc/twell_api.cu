@@ -42,31 +42,6 @@ int sm_count() {
   return cache[dev];
 }
 
-bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool valid_tile(int tile_w) { return tile_w == 32 || tile_w == 64 || tile_w == 128 || tile_w == 256; }
-
-// Shape rules shared by every call.
-twell_status check_shape(int M, int d_ff, int tile_w, int ell_w) {
-  if (M < 0 || d_ff <= 0 || !valid_tile(tile_w) || d_ff % tile_w != 0) return TWELL_ERR_INVALID_ARG;
-  if (ell_w < 1 || ell_w > tile_w) return TWELL_ERR_INVALID_ARG;
-  return TWELL_OK;
-}
-
-twell_status check_matrix(const twell_matrix *a, int M, int d_ff, int tile_w, int ell_w) {
-  if (a == nullptr) return TWELL_ERR_INVALID_ARG;
-  if (a->M != M || a->d_ff != d_ff || a->tile_w != tile_w || a->ell_w != ell_w)
-    return TWELL_ERR_INVALID_ARG;
-  if (a->ovf_capacity < 0 || a->n_ovf == nullptr || a->status == nullptr) return TWELL_ERR_INVALID_ARG;
-  if (M > 0 && (a->vals == nullptr || a->idx == nullptr || a->nnz == nullptr)) return TWELL_ERR_INVALID_ARG;
-  if (!a16(a->vals) || !a16(a->idx) || !a16(a->nnz)) return TWELL_ERR_INVALID_ARG;
-  if (a->ovf_capacity > 0 && (a->ovf_pos == nullptr || a->ovf_dense == nullptr)) return TWELL_ERR_INVALID_ARG;
-  if (!a16(a->ovf_pos) || !a16(a->ovf_dense)) return TWELL_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(a->n_ovf) & 3u) || (reinterpret_cast<uintptr_t>(a->status) & 3u))
-    return TWELL_ERR_INVALID_ARG;
-  return TWELL_OK;
-}
-
 // Workspace regions: overflow staging + per-block path flags.
 struct Ws {
   WsLayout L;
@@ -295,6 +270,40 @@ TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int cap_tok) {
 
 }  // namespace
 
+bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_tile(int tile_w) { return tile_w == 32 || tile_w == 64 || tile_w == 128 || tile_w == 256; }
+
+// Shape rules shared by every call.
+twell_status check_shape(int M, int d_ff, int tile_w, int ell_w) {
+  if (M < 0 || d_ff <= 0 || !valid_tile(tile_w) || d_ff % tile_w != 0) return TWELL_ERR_INVALID_ARG;
+  if (ell_w < 1 || ell_w > tile_w) return TWELL_ERR_INVALID_ARG;
+  return TWELL_OK;
+}
+
+twell_status check_matrix(const twell_matrix *a, int M, int d_ff, int tile_w, int ell_w) {
+  if (a == nullptr) return TWELL_ERR_INVALID_ARG;
+  if (a->M != M || a->d_ff != d_ff || a->tile_w != tile_w || a->ell_w != ell_w)
+    return TWELL_ERR_INVALID_ARG;
+  if (a->ovf_capacity < 0 || a->n_ovf == nullptr || a->status == nullptr) return TWELL_ERR_INVALID_ARG;
+  if (M > 0 && (a->vals == nullptr || a->idx == nullptr || a->nnz == nullptr)) return TWELL_ERR_INVALID_ARG;
+  if (!a16(a->vals) || !a16(a->idx) || !a16(a->nnz)) return TWELL_ERR_INVALID_ARG;
+  if (a->ovf_capacity > 0 && (a->ovf_pos == nullptr || a->ovf_dense == nullptr)) return TWELL_ERR_INVALID_ARG;
+  if (!a16(a->ovf_pos) || !a16(a->ovf_dense)) return TWELL_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a->n_ovf) & 3u) || (reinterpret_cast<uintptr_t>(a->status) & 3u))
+    return TWELL_ERR_INVALID_ARG;
+  return TWELL_OK;
+}
+
+twell_status check_pack_args(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
+                             const twell_matrix *out) {
+  twell_status st = check_shape(M, d_ff, tile_w, ell_w);
+  if (st != TWELL_OK) return st;
+  if (M == 0) return TWELL_OK;   // documented no-op: nothing is read or written
+  if (h == nullptr || !a16(h) || ld_h < d_ff || ld_h % 8 != 0) return TWELL_ERR_INVALID_ARG;
+  return check_matrix(out, M, d_ff, tile_w, ell_w);
+}
+
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                               uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle, CUtensorMapDataType dtype) {
@@ -339,15 +348,10 @@ size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w
 
 twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
                         const twell_matrix *out, void *ws, size_t ws_bytes, void *stream) {
-  twell_status st = check_shape(M, d_ff, tile_w, ell_w);
-  if (st != TWELL_OK) return st;
-  if (M == 0) return TWELL_OK;   // documented no-op: nothing is read or written
-  if (h == nullptr || !a16(h) || ld_h < d_ff || ld_h % 8 != 0) return TWELL_ERR_INVALID_ARG;
-  st = check_matrix(out, M, d_ff, tile_w, ell_w);
-  if (st != TWELL_OK) return st;
+  twell_status st = check_pack_args(h, M, d_ff, ld_h, tile_w, ell_w, out);
+  if (st != TWELL_OK || M == 0) return st;
   st = check_ws(ws, ws_bytes, M, d_ff, tile_w, out->ovf_capacity);
   if (st != TWELL_OK) return st;
-  if (M == 0) return TWELL_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const PackTarget t = make_target(out, ws);
   st = reset_for_pack(t, s);

@@ -53,6 +53,17 @@ struct TwellView {
   int32_t *status;
 };
 
+// Argument rules shared by the entry points (twell_api.cu).  Each returns
+// TWELL_OK or the status the call reports; none touches the GPU.
+bool a16(const void *p);                 // 16-byte aligned (NULL passes)
+bool valid_tile(int tile_w);
+twell_status check_shape(int M, int d_ff, int tile_w, int ell_w);
+twell_status check_matrix(const twell_matrix *a, int M, int d_ff, int tile_w, int ell_w);
+// twell_pack's rules without the workspace: shape, then (M > 0) h and the
+// destination matrix.  M == 0 returns TWELL_OK before `h` and `out` are read.
+twell_status check_pack_args(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
+                             const twell_matrix *out);
+
 // Workspace carve-up (every region 256-byte aligned).
 struct WsLayout {
   size_t ctr, row_ovf, row_prefix, stage_pos, stage_dense, total;

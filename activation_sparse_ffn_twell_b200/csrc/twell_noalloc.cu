@@ -47,8 +47,6 @@ cudaError_t scratch_address(void **out) {
   return cudaSuccess;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace twell
 
@@ -57,22 +55,9 @@ using namespace twell;
 extern "C" twell_status twell_pack_noalloc(const uint16_t *h, int M, int d_ff, int ld_h,
                                            int tile_w, int ell_w, const twell_matrix *out,
                                            void *stream) {
-  // -- same shape and pointer rules as twell_pack
-  if (M < 0 || d_ff <= 0 || !(tile_w == 32 || tile_w == 64 || tile_w == 128 || tile_w == 256) ||
-      d_ff % tile_w != 0 || ell_w < 1 || ell_w > tile_w)
-    return TWELL_ERR_INVALID_ARG;
-  if (out == nullptr || out->M != M || out->d_ff != d_ff || out->tile_w != tile_w ||
-      out->ell_w != ell_w || out->ovf_capacity < 0 || out->n_ovf == nullptr ||
-      out->status == nullptr)
-    return TWELL_ERR_INVALID_ARG;
-  if (M == 0) return TWELL_OK;
-  if (h == nullptr || !aligned16(h) || ld_h < d_ff || ld_h % 8 != 0) return TWELL_ERR_INVALID_ARG;
-  if (out->vals == nullptr || out->idx == nullptr || out->nnz == nullptr || !aligned16(out->vals) ||
-      !aligned16(out->idx) || !aligned16(out->nnz))
-    return TWELL_ERR_INVALID_ARG;
-  if (out->ovf_capacity > 0 && (out->ovf_pos == nullptr || out->ovf_dense == nullptr ||
-                                !aligned16(out->ovf_pos) || !aligned16(out->ovf_dense)))
-    return TWELL_ERR_INVALID_ARG;
+  // -- the same argument rules as twell_pack (shared code, so the two cannot drift)
+  const twell_status st = check_pack_args(h, M, d_ff, ld_h, tile_w, ell_w, out);
+  if (st != TWELL_OK || M == 0) return st;
 
   // -- the scratch this call needs must fit the fixed array
   const WsLayout L = ws_layout(M, tile_w, out->ovf_capacity);

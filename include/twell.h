@@ -183,7 +183,12 @@ twell_status twell_ffn_forward(const uint16_t *x, const uint16_t *W_up, const ui
  *     allows ovf_capacity up to about 15,900).
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current).  Make that first call before any CUDA
- *     stream capture.
+ *     stream capture.  The address is kept for the life of the process and
+ *     belongs to the device's primary context: do not call this entry point
+ *     after cudaDeviceReset on that device, nor from a non-primary driver
+ *     context.
+ *   - Arguments are checked by the same code as twell_pack's, with the same
+ *     results; M == 0 is a no-op that reads neither `h` nor `out`.
  *   - All calls share the one array and it keeps the previous call's contents;
  *     each call clears what must start at zero.  Calls whose executions overlap
  *     on the GPU (different streams, or different host threads, without ordering

@@ -136,3 +136,34 @@ def test_no_gpu_means_cuda_error_not_a_crash(L):
     h = 0x8000000
     r = L.twell_pack(h, 256, 1024, 1024, 128, 16, ctypes.byref(m), 0x9000000, 1 << 30, None)
     assert r == 4
+
+
+def test_pack_noalloc_argument_rules_match_pack(L):
+    """twell_pack_noalloc shares twell_pack's validators: the same inputs are
+    rejected on the host with the same status, before any launch."""
+    import activation_sparse_ffn_twell_b200 as T
+    bp = ctypes.byref
+    ws, wsb = 0x9000000, 1 << 30
+    h = 0x8000000
+
+    def both(hh, M, f, ld, tw, E, m):
+        a = L.twell_pack(hh, M, f, ld, tw, E, m, ws, wsb, None)
+        b = L.twell_pack_noalloc(hh, M, f, ld, tw, E, m, None)
+        assert a == b, (a, b)
+        return b
+
+    m = _matrix()
+    assert both(h + 2, 256, 1024, 1024, 128, 16, bp(m)) == 1              # misaligned h
+    assert both(h, 256, 1024, 1000, 128, 16, bp(m)) == 1                  # ld_h < d_ff
+    assert both(h, 256, 1024, 1024, 100, 16, bp(m)) == 1                  # tile_w
+    assert both(h, 256, 1024, 1024, 128, 16, None) == 1                   # no matrix
+    assert both(h, 256, 1024, 1024, 128, 16, bp(_matrix(M=128))) == 1    # M mismatch
+    # a misaligned device status word or overflow counter would be written by
+    # the kernels as int32: both entry points reject it
+    for field in ("n_ovf", "status"):
+        bad = _matrix()
+        setattr(bad, field, getattr(bad, field) + 2)
+        assert both(h, 256, 1024, 1024, 128, 16, bp(bad)) == 1
+    # M == 0 is a no-op for both, even without a destination
+    assert both(h, 0, 1024, 1024, 128, 16, None) == 0
+    assert both(None, 0, 1024, 1024, 128, 16, bp(_matrix(M=0))) == 0
