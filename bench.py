@@ -188,12 +188,21 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def fused():
+        T.twell_ffn_forward(x, wu, b, wd, tile_w=tw, ell_w=E, W_gate=wg, mode=args.mode, out=a, y=y)
+
+    def split():
         T.twell_up_pack(x, wu, b, wg, tile_w=tw, ell_w=E, out=a)
         T.twell_spmm(a, wd, mode=args.mode, y=y)
 
+    # warm-up: the timed call itself (W steps), then the phase calls of the
+    # second loop, so neither loop's first step pays for first use
     for _ in range(args.warmup):
-        step()
+        flush.zero_()
+        fused()
+    for _ in range(3):
+        flush.zero_()
+        split()
     code, n_ovf = T.read_status(a)
     if code != 0:
         raise SystemExit(f"status {T.STATUS[code]} after warm-up")
@@ -221,8 +230,7 @@ def run_ours(args):
             flush.zero_()                      # evict L2 between steps (inputs < 126 MB)
             e0, e1 = ev[i]
             e0.record(stream)
-            T.twell_ffn_forward(x, wu, b, wd, tile_w=tw, ell_w=E, W_gate=wg, mode=args.mode,
-                                out=a, y=y)
+            fused()
             e1.record(stream)
         torch.cuda.synchronize(dev)
         wall = time.perf_counter() - wall0
@@ -236,7 +244,11 @@ def run_ours(args):
             e2.record(stream)
         torch.cuda.synchronize(dev)
     D.barrier(dev)
-    step_ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / args.steps
+    # the step time is the median of the K per-step event intervals (robust to a
+    # stray slow step); the mean is reported beside it
+    step_all = [e0.elapsed_time(e1) for e0, e1 in ev]
+    step_ms = _median(step_all)
+    step_mean = sum(step_all) / len(step_all)
     up_ms = [e0.elapsed_time(e1) for e0, e1, _ in evp]
     down_ms = [e1.elapsed_time(e2) for _, e1, e2 in evp]
     step_ms_max = D.max_over_ranks(step_ms, dev if world > 1 and args.gpus > 1 else None)
@@ -245,8 +257,8 @@ def run_ours(args):
         raise SystemExit(f"status {T.STATUS[code]} in timed region")
 
     tokens_s = world * M / (step_ms_max * 1e-3)
-    up_s = sum(up_ms) / len(up_ms) * 1e-3
-    down_s = sum(down_ms) / len(down_ms) * 1e-3
+    up_s = _median(up_ms) * 1e-3
+    down_s = _median(down_ms) * 1e-3
     rl = _roofline_layer(L, nnz_total, touched, peaks)
     # Per-phase rooflines from algorithmic work: each phase is bound by the
     # slower of its FLOPs at the tensor peak and its unavoidable bytes at the HBM
@@ -293,6 +305,9 @@ def run_ours(args):
     result = {
         "metric": METRIC, "value": tokens_s, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+        "ms_per_step_stat": f"median of {args.steps} CUDA-event step intervals",
+        "ms_per_step_mean": step_mean, "ms_per_step_min": min(step_all),
+        "phase_sum_ms": (up_s + down_s) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded N(0,1/fan_in) weights, bias for target density)",
         "config": {"workload": {"relu_15b": "relu_ffn_layer_1.5b"}.get(args.workload, args.workload),
@@ -322,8 +337,11 @@ def run_ours(args):
     if not args.quick:
         result["dense_ffn"] = _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg)
         result["e2e"] = _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world)
-        if args.sweep:
-            result["density_sweep"] = _sweep(T, args, dev, peaks)
+        if args.workload == "relu_15b":
+            # fused layer against the dense cuBLAS FFN at every density of the
+            # 1.5B-layer workload (--sweep adds the forced gather / MMA paths)
+            result["density_sweep"] = _sweep(T, args, dev, peaks,
+                                             modes=("auto", "gather", "mma") if args.sweep else ("auto",))
     if args.backward and not L.gated and M % 128 == 0:
         result["backward"] = _backward(T, x, wu, b, wd, a, args, flush, stream, dev)
     if args.token_overflow:
@@ -336,6 +354,12 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
     del a
     D.finish()
+
+
+def _median(v):
+    s = sorted(v)
+    n = len(s)
+    return s[n // 2] if n % 2 else 0.5 * (s[n // 2 - 1] + s[n // 2])
 
 
 def _touched_rows(a, torch):
@@ -402,7 +426,7 @@ def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):
         e1.record(stream)
         ts.append((e0, e1))
     torch.cuda.synchronize(dev)
-    ms = sum(a.elapsed_time(b) for a, b in ts) / len(ts)
+    ms = _median([a.elapsed_time(b) for a, b in ts])
     return {"ms_per_step": ms, "tokens_s": x.shape[0] / (ms * 1e-3),
             "impl": "torch.matmul bf16 (cuBLAS): relu(x W_up^T + b) W_down"}
 
@@ -557,13 +581,37 @@ def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
                      "upload / layer / download pipelined on three streams")}
 
 
-def _sweep(T, args, dev, peaks):
+SWEEP_DENSITIES = (0.20, 0.10, 0.05, 0.02, 0.01)
+
+
+def _sweep(T, args, dev, peaks, modes=("auto",)):
+    """The 1.5B-scale layer at each target density: the fused twell_ffn_forward
+    (per down mode in `modes`) and the same-shape dense cuBLAS FFN, timed in the
+    same run the same way (median of CUDA-event step intervals, L2 flushed
+    between steps), with the layer roofline and the margin over dense."""
     import numpy as np
     import torch
     import torch.nn.functional as F
     out = []
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    for rho in (0.20, 0.10, 0.05, 0.01):
+    n_steps = max(10, min(args.steps, 30))
+
+    def timed(fn):
+        for _ in range(3):
+            flush.zero_()
+            fn()
+        evs = []
+        for _ in range(n_steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        return _median([p.elapsed_time(q) for p, q in evs])
+
+    for rho in SWEEP_DENSITIES:
         L = _workload(rho, args.M, args.seed)
         tb = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
         x, wu, b, wd = tb(L.x), tb(L.w_up), tb(L.b), tb(L.w_down)
@@ -571,62 +619,44 @@ def _sweep(T, args, dev, peaks):
         a = T.TwELL.allocate(L.M, L.d_ff, L.tile_w, L.ell_w, T.default_ovf_capacity(L.M, T_tiles),
                              device=dev)
         y = torch.empty((L.M, L.d_model), dtype=torch.bfloat16, device=dev)
-        row = {"target_density": rho, "ell_w": L.ell_w}
-        for mode in ("auto", "gather", "mma"):
-            for _ in range(3):
-                T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=mode, out=a, y=y)
-            evs = []
-            for _ in range(max(5, args.steps // 4)):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode=mode, out=a, y=y)
-                e1.record()
-                evs.append((e0, e1))
-            torch.cuda.synchronize(dev)
-            row[f"{mode}_ms"] = sum(p.elapsed_time(q) for p, q in evs) / len(evs)
+        row = {"target_density": rho, "ell_w": L.ell_w, "steps": n_steps}
+        for mode in modes:
+            row[f"{mode}_ms"] = timed(lambda: T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w,
+                                                                  ell_w=L.ell_w, mode=mode, out=a, y=y))
+        T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w, mode="auto", out=a, y=y)
         code, n_ovf = T.read_status(a)
+        if code != 0:
+            raise SystemExit(f"sweep {rho}: status {T.STATUS[code]}")
         nnz_total = int(a.nnz_u16().sum().item())
         row["measured_density"] = nnz_total / float(L.M * L.d_ff)
         row["n_ovf"] = n_ovf
         rl = _roofline_layer(L, nnz_total, int(_touched_rows(a, torch).item()), peaks)
-        best = min(row["auto_ms"], row["gather_ms"], row["mma_ms"])
         row["roofline_ms"] = rl["t_s"] * 1e3
         row["frac_roofline_auto"] = rl["t_s"] * 1e3 / row["auto_ms"]
         row["tokens_s_auto"] = L.M / (row["auto_ms"] * 1e-3)
-        # dense comparator
-        for _ in range(3):
-            torch.matmul(torch.relu(F.linear(x, wu, b)), wd)
-        evs = []
-        for _ in range(max(5, args.steps // 4)):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            torch.matmul(torch.relu(F.linear(x, wu, b)), wd)
-            e1.record()
-            evs.append((e0, e1))
-        torch.cuda.synchronize(dev)
-        row["dense_ms"] = sum(p.elapsed_time(q) for p, q in evs) / len(evs)
+        row["dense_ms"] = timed(lambda: torch.matmul(torch.relu(F.linear(x, wu, b)), wd))
         row["speedup_vs_dense_auto"] = row["dense_ms"] / row["auto_ms"]
-        row["best_ms"] = best
+        row["margin_vs_dense_auto"] = 1.0 - row["auto_ms"] / row["dense_ms"]
         out.append(row)
         del a, x, wu, b, wd, y
+        torch.cuda.empty_cache()
     return out
 
 
 # ---------------------------------------------------------------------------
-def _cpu_baseline(L, seconds=10.0, sample_tokens=256):
-    """The oracle, as it stands, on the host cores over a bounded token sample of
-    the same layer (full weights); repeats the sample until ~`seconds` elapse."""
-    import numpy as np
-    import oracle as O
+def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+        return max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count()
-    done, t0 = 0, time.perf_counter()
-    reps = 0
+        return os.cpu_count()
+
+
+def _oracle_rate(L, seconds, sample_tokens, max_reps=64):
+    """Tokens/s of the oracle forward over repeated `sample_tokens`-token slices
+    of the batch (full weights) until ~`seconds` elapse.  Returns (rate, reps, s)."""
+    import oracle as O
+    done, reps, t0 = 0, 0, time.perf_counter()
     while True:
         r0 = (reps * sample_tokens) % L.M
         rows = slice(r0, r0 + sample_tokens)
@@ -634,37 +664,79 @@ def _cpu_baseline(L, seconds=10.0, sample_tokens=256):
         done += min(sample_tokens, L.M - r0)
         reps += 1
         el = time.perf_counter() - t0
-        if el >= seconds or reps >= 64:
+        if el >= seconds or reps >= max_reps:
+            return done / el, reps, el
+
+
+def _cpu_baseline(L, seconds=10.0, sample_tokens=256):
+    """The oracle, as it stands, on the host cores over a bounded token sample of
+    the same layer (full weights): the whole forward on every BLAS thread, the
+    same on one core, and the reference packer alone."""
+    import oracle as O
+    threads = _blas_threads()
+    rate, reps, el = _oracle_rate(L, seconds, sample_tokens)
+    out = {"value": rate, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+           "sample": f"{reps} x {sample_tokens}-token slices of the {L.M}-token batch, full "
+                     f"{L.d_model}x{L.d_ff} weights, fp64 NumPy, {el:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            r1, reps1, el1 = _oracle_rate(L, max(1.0, seconds / 4), 64, max_reps=16)
+        out["value_1core"] = r1
+        out["sample_1core"] = f"{reps1} x 64-token slices on 1 core, {el1:.1f} s"
+    except Exception as e:   # threadpoolctl missing: say so rather than guess
+        out["value_1core"] = None
+        out["sample_1core"] = f"unavailable: {type(e).__name__}"
+    # packer alone: the reference TwELL packer on the sample's (untimed) h
+    h = O.hidden(L.x[:sample_tokens], L.w_up, L.b, L.w_gate)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        O.twell_pack(h, L.tile_w, L.ell_w)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= max(0.5, seconds / 8) or n >= 64:
             break
-    return {"value": done / el, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": f"{reps} x {sample_tokens}-token slices of the {L.M}-token batch, full "
-                      f"{L.d_model}x{L.d_ff} weights, fp64 NumPy, {el:.1f} s"}
+    out["pack_tokens_s"] = n * h.shape[0] / el
+    out["sample_pack"] = f"{n} packs of a {h.shape[0]}-token h, {el:.1f} s"
+    return out
 
 
 def run_reference(args):
-    """--impl reference: the CPU oracle timed on the host cores (rank 0 only)."""
+    """--impl reference: the CPU oracle timed on the host cores (rank 0 only).
+    Each step is the oracle forward over a `ref_tokens`-token sample of the
+    batch; ms_per_step is that step's measured time (not scaled to the batch)."""
     from activation_sparse_ffn_twell_b200 import dist as D
     rank, _, world = D.env_rank_world()
     if rank != 0:
         return
+    import oracle as O
     L = _workload(args.density, args.M, args.seed)
-    for _ in range(args.warmup):
-        _cpu_baseline(L, seconds=0.0, sample_tokens=64)
-    per = []
-    for _ in range(args.steps):
-        cb = _cpu_baseline(L, seconds=0.0, sample_tokens=args.ref_tokens)
-        per.append(cb)
-    value = sum(c["value"] for c in per) / len(per)
-    ms = args.ref_tokens / value * 1e3 * (L.M / args.ref_tokens)
+    n = args.ref_tokens
+
+    def one(r0):
+        rows = slice(r0 % L.M, r0 % L.M + n)
+        t0 = time.perf_counter()
+        O.ffn_forward(L.x[rows], L.w_up, L.b, L.w_down, L.tile_w, L.ell_w, L.w_gate)
+        return time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        one(i * n)
+    per = [one((args.warmup + i) * n) for i in range(args.steps)]
+    ms = _median(per) * 1e3
+    value = n / (ms * 1e-3)
+    cores = _blas_threads()
     print(json.dumps({
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "impl": "reference", "device": "cpu (host cores)",
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "impl": "reference",
+        "device": "cpu (host cores)", "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "ms_per_step_stat": f"median of {args.steps} measured steps",
+        "total_timed_s": sum(per), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "relu_ffn_layer_1.5b", "M": L.M, "d_model": L.d_model,
-                   "d_ff": L.d_ff, "target_density": args.density, "tile_w": L.tile_w,
-                   "ell_w": L.ell_w},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per[0]["cores"], "kind": "oracle",
-                         "sample": f"each step: {args.ref_tokens} tokens of the {L.M}-token batch"},
+        "config": {"workload": "relu_ffn_layer_1.5b", "M": L.M, "tokens_per_step": n,
+                   "d_model": L.d_model, "d_ff": L.d_ff, "target_density": args.density,
+                   "tile_w": L.tile_w, "ell_w": L.ell_w},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the oracle forward over {n} tokens of the "
+                                   f"{L.M}-token batch (full weights); ms_per_step is that time"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

@@ -25,6 +25,24 @@ def test_reference_arm_prints_the_contract_line():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "relu_ffn_layer_1.5b"
+    # the step time is what was measured for the sampled tokens, not scaled up
+    assert line["config"]["tokens_per_step"] == 16
+    assert line["ms_per_step"] <= 1e3 * line["total_timed_s"] * 1.0001
+    assert abs(line["value"] - 16 / (line["ms_per_step"] * 1e-3)) < 1e-6 * line["value"]
+
+
+def test_cpu_baseline_reports_all_cores_one_core_and_the_packer():
+    import twell_synth as S
+    L = S.tiny_relu(0)
+    cb = bench._cpu_baseline(L, seconds=0.2, sample_tokens=32)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] >= 1
+    assert cb["value_1core"] is None or cb["value_1core"] > 0
+    assert cb["pack_tokens_s"] > 0 and "pack" in cb["sample_pack"]
+
+
+def test_median():
+    assert bench._median([3.0, 1.0, 2.0]) == 2.0
+    assert bench._median([4.0, 1.0, 2.0, 3.0]) == 2.5
 
 
 def test_traffic_lookup_follows_the_kernel_source(monkeypatch, tmp_path):
