@@ -34,7 +34,7 @@ _LIB_PATH = os.path.join(_HERE, "libtwell_b200.so")
 STATUS = {0: "TWELL_OK", 1: "TWELL_ERR_INVALID_ARG", 2: "TWELL_ERR_UNSUPPORTED",
           3: "TWELL_ERR_OVERFLOW_CAPACITY", 4: "TWELL_ERR_CUDA", 5: "TWELL_ERR_TIMEOUT",
           6: "TWELL_ERR_WORKSPACE"}
-DOWN_MODES = {"auto": 0, "gather": 1, "mma": 2}
+DOWN_MODES = {"auto": 0, "gather": 1, "mma": 2, "sparse": 3}
 
 
 class TwellError(RuntimeError):

@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) k_spmm_gather(TwellView A, const uint16_t
        it < items; it += static_cast<long long>(gridDim.x) * warps_per_cta) {
     const int r = static_cast<int>(it / passes);
     const int pass = static_cast<int>(it - static_cast<long long>(r) * passes);
-    if (blk_path != nullptr && blk_path[r / kBlockM] != 0) continue;   // owned by the MMA path
+    if (blk_path != nullptr && blk_path[r / kBlockM] != kPathGather) continue;   // a tensor-core path's
     const int col_base = pass * cols_per_pass + lane * 8;
 
     float acc[NCH][8];

@@ -94,7 +94,7 @@ __device__ __forceinline__ int find_ovf(const int32_t *pos, int n, int key) {
 }
 
 __device__ __forceinline__ bool tile_owned(const DownParams &P, int m_blk) {
-  return P.blk_path == nullptr || P.blk_path[m_blk] != 0;
+  return P.blk_path == nullptr || P.blk_path[m_blk] == kPathDense;
 }
 
 // The schedule helpers below also compile for the host, where

@@ -47,21 +47,28 @@ struct Ws {
   WsLayout L;
   size_t blk_path;   // [M / 128 + 1] i32: down path of each 128-token block
   size_t l1_part;    // [M][T] fp32: per (token, tile) sums of |h| (statistics)
-  size_t split;      // split schedule of the tensor-core down-projection (last;
-                     // present when d_model is given and the shape can use it)
+  size_t split;      // split schedule of the tensor-core down-projection (present
+                     // when d_model is given and the shape can use it)
   size_t split_bytes;
+  size_t sp;         // excess lists of the 2:4 down path (present when d_model is
+                     // given and the shape can use it)
+  size_t sp_bytes;
   size_t total;
 };
 
 // d_model = 0: the regions of the calls that never run the down-projection.
-Ws ws_plan(int M, int d_ff, int tile_w, int cap, int d_model = 0) {
+Ws ws_plan(int M, int d_ff, int tile_w, int ell_w, int cap, int d_model = 0) {
   Ws w;
   w.L = ws_layout(M, tile_w, cap);
   w.blk_path = w.L.total;
   w.l1_part = align256(w.blk_path + sizeof(int32_t) * static_cast<size_t>((M + kBlockM - 1) / kBlockM + 1));
   w.split = align256(w.l1_part + sizeof(float) * static_cast<size_t>(M) * (d_ff / tile_w));
   w.split_bytes = d_model > 0 ? split_ws_bytes(M, d_model) : 0;
-  w.total = align256(w.split + w.split_bytes);
+  w.sp = align256(w.split + w.split_bytes);
+  TwellView v = {};
+  v.M = M; v.f = d_ff; v.tw = tile_w; v.E = ell_w; v.T = d_ff / tile_w;
+  w.sp_bytes = (d_model > 0 && sp_eligible(v, d_model)) ? sp_ws_bytes(M, d_ff, d_model) : 0;
+  w.total = align256(w.sp + w.sp_bytes);
   return w;
 }
 
@@ -78,7 +85,7 @@ SplitWs split_ptrs(const Ws &w, void *ws) {
 }
 
 PackTarget make_target(const twell_matrix *a, void *ws) {
-  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity);
+  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ell_w, a->ovf_capacity);
   uint8_t *base = static_cast<uint8_t *>(ws);
   PackTarget t;
   t.M = a->M; t.f = a->d_ff; t.tw = a->tile_w; t.E = a->ell_w; t.T = a->d_ff / a->tile_w;
@@ -110,8 +117,8 @@ twell_status reset_for_pack(const PackTarget &t, cudaStream_t s) {
   return from_cuda(launch_pack_reset(t, s));
 }
 
-twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int cap, int d_model = 0) {
-  const Ws w = ws_plan(M, d_ff, tile_w, cap, d_model);
+twell_status check_ws(void *ws, size_t ws_bytes, int M, int d_ff, int tile_w, int ell_w, int cap, int d_model = 0) {
+  const Ws w = ws_plan(M, d_ff, tile_w, ell_w, cap, d_model);
   if (ws == nullptr || !a16(ws) || ws_bytes < w.total) return TWELL_ERR_WORKSPACE;
   return TWELL_OK;
 }
@@ -127,7 +134,7 @@ twell_status up_pack_checked(const uint16_t *x, const uint16_t *W_up, const uint
   if (sms <= 0) return TWELL_ERR_CUDA;
   twell_status st = reset_for_pack(t, s);
   if (st != TWELL_OK) return st;
-  const Ws w = ws_plan(M, d_ff, tile_w, out->ovf_capacity);
+  const Ws w = ws_plan(M, d_ff, tile_w, ell_w, out->ovf_capacity);
   float *l1_part = (l1 != nullptr) ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + w.l1_part)
                                    : nullptr;
   UpArgs a;
@@ -156,7 +163,7 @@ twell_status validate_up(const uint16_t *x, const uint16_t *W_up, const uint16_t
   if (st != TWELL_OK) return st;
   if (ell_w > kMaxEllFused) return TWELL_ERR_UNSUPPORTED;
   if (W_gate != nullptr && tile_w > 128) return TWELL_ERR_UNSUPPORTED;
-  return check_ws(ws, ws_bytes, M, d_ff, tile_w, out->ovf_capacity);
+  return check_ws(ws, ws_bytes, M, d_ff, tile_w, ell_w, out->ovf_capacity);
 }
 
 twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_model, uint16_t *y,
@@ -165,16 +172,14 @@ twell_status validate_spmm(const twell_matrix *a, const uint16_t *W_down, int d_
   twell_status st = check_shape(a->M, a->d_ff, a->tile_w, a->ell_w);
   if (st != TWELL_OK) return st;
   if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
-  if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
+  if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA && mode != TWELL_DOWN_SPARSE)
     return TWELL_ERR_INVALID_ARG;
   if (a->M == 0) return TWELL_OK;   // documented no-op
   st = check_matrix(a, a->M, a->d_ff, a->tile_w, a->ell_w);
   if (st != TWELL_OK) return st;
   if (d_model <= 0 || d_model % 64 != 0) return TWELL_ERR_INVALID_ARG;
   if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y)) return TWELL_ERR_INVALID_ARG;
-  if (mode != TWELL_DOWN_AUTO && mode != TWELL_DOWN_GATHER && mode != TWELL_DOWN_MMA)
-    return TWELL_ERR_INVALID_ARG;
-  return check_ws(ws, ws_bytes, a->M, a->d_ff, a->tile_w, a->ovf_capacity, d_model);
+  return check_ws(ws, ws_bytes, a->M, a->d_ff, a->tile_w, a->ell_w, a->ovf_capacity, d_model);
 }
 
 // pdl_first: the call's first kernel may be a dependent launch (true only when
@@ -191,9 +196,23 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
   // decode-size batches: the split-K tensor-core kernel streams W_down over every SM
   if (decode_down_eligible(a->M))
     return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, pdl_first, s));
-  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ovf_capacity, d_model);
+  const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ell_w, a->ovf_capacity, d_model);
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
   const SplitWs sp = split_ptrs(w, ws);
+  if (mode == TWELL_DOWN_SPARSE && w.sp_bytes > 0) {
+    // 2:4 structured-sparse path (explicit mode only: on B200 it measured
+    // slower than the dense tensor-core path at every density, see the path's
+    // kernel file): the prep pass builds the 2:4 operand and every token's
+    // excess product, the decision pass gives each 256-token group its path,
+    // and the 2:4 and dense kernels each take their own groups.
+    void *spb = static_cast<uint8_t *>(ws) + w.sp;
+    cudaError_t e = launch_sp_prep(v, W_down, d_model, spb, -1.0f, true, blk, sp.ctr, pdl_first, s);
+    if (e != cudaSuccess) return TWELL_ERR_CUDA;
+    e = launch_spmm_sp(v, W_down, d_model, y, blk, spb, sms, true, s);
+    if (e != cudaSuccess) return TWELL_ERR_CUDA;
+    return from_cuda(launch_spmm_mma(v, W_down, d_model, y, blk, sp, sms, true, s));
+  }
+  if (mode == TWELL_DOWN_SPARSE) mode = TWELL_DOWN_MMA;   // shape not eligible: dense tensor-core path
   // The block pass also zeroes the split schedule's counters.  MMA mode hands
   // the tensor-core kernel no block flags: its W_down stream starts before the
   // kernel waits for its predecessor, and with no gather launch in between that
@@ -237,7 +256,8 @@ BwLayout bw_layout(int M, int d_model, int d_ff, int tile_w, int ell_w, int cap,
   b.db_part = take(4 * F * Tt);
   b.stage_L = ws_layout(d_ff, 128, cap_t);
   b.stage = take(b.stage_L.total);
-  const size_t s1 = ws_plan(M, d_ff, tile_w, cap, d_model).total, s2 = ws_plan(d_ff, M, 128, cap_t, d_model).total;
+  const size_t s1 = ws_plan(M, d_ff, tile_w, ell_w, cap, d_model).total,
+               s2 = ws_plan(d_ff, M, 128, ell_t, cap_t, d_model).total;
   b.spmm = take(s1 > s2 ? s1 : s2);
   b.total = o;
   return b;
@@ -248,7 +268,7 @@ struct TokLayout {
   size_t flag, rank, main_nnz, tok_pos, d_vals, d_idx, d_nnz, y_dense, words, spmm, total;
 };
 
-TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int cap_tok) {
+TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int ell_w, int cap_tok) {
   TokLayout L;
   const size_t T = d_ff / tile_w;
   size_t o = 0;
@@ -262,7 +282,8 @@ TokLayout tok_layout(int M, int d_model, int d_ff, int tile_w, int cap_tok) {
   L.d_nnz = take(2 * static_cast<size_t>(cap_tok) * T);
   L.y_dense = take(2 * static_cast<size_t>(cap_tok) * d_model);
   L.words = take(64);
-  const size_t s1 = ws_plan(M, d_ff, tile_w, 0, d_model).total, s2 = ws_plan(cap_tok, d_ff, tile_w, 0, d_model).total;
+  const size_t s1 = ws_plan(M, d_ff, tile_w, ell_w, 0, d_model).total,
+               s2 = ws_plan(cap_tok, d_ff, tile_w, tile_w, 0, d_model).total;
   L.spmm = take(s1 > s2 ? s1 : s2);
   L.total = o;
   return L;
@@ -324,7 +345,7 @@ using namespace twell;
 
 extern "C" {
 
-int twell_version(void) { return 200; }
+int twell_version(void) { return 300; }
 
 const char *twell_status_string(twell_status s) {
   switch (s) {
@@ -343,14 +364,14 @@ size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w
                              int ovf_capacity) {
   if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || ovf_capacity < 0) return 0;
   if (d_model <= 0 || d_model % 64 != 0 || (gated != 0 && gated != 1)) return 0;
-  return ws_plan(M, d_ff, tile_w, ovf_capacity, d_model).total;
+  return ws_plan(M, d_ff, tile_w, ell_w, ovf_capacity, d_model).total;
 }
 
 twell_status twell_pack(const uint16_t *h, int M, int d_ff, int ld_h, int tile_w, int ell_w,
                         const twell_matrix *out, void *ws, size_t ws_bytes, void *stream) {
   twell_status st = check_pack_args(h, M, d_ff, ld_h, tile_w, ell_w, out);
   if (st != TWELL_OK || M == 0) return st;
-  st = check_ws(ws, ws_bytes, M, d_ff, tile_w, out->ovf_capacity);
+  st = check_ws(ws, ws_bytes, M, d_ff, tile_w, ell_w, out->ovf_capacity);
   if (st != TWELL_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const PackTarget t = make_target(out, ws);
@@ -494,7 +515,7 @@ size_t twell_token_overflow_workspace_bytes(int M, int d_model, int d_ff, int ti
                                             int cap_tok) {
   if (check_shape(M, d_ff, tile_w, ell_w) != TWELL_OK || cap_tok < 1) return 0;
   if (d_model <= 0 || d_model % 64 != 0) return 0;
-  return tok_layout(M, d_model, d_ff, tile_w, cap_tok).total;
+  return tok_layout(M, d_model, d_ff, tile_w, ell_w, cap_tok).total;
 }
 
 twell_status twell_spmm_token_overflow(const twell_matrix *a, const uint16_t *W_down, int d_model,
@@ -510,7 +531,7 @@ twell_status twell_spmm_token_overflow(const twell_matrix *a, const uint16_t *W_
   if (W_down == nullptr || y == nullptr || !a16(W_down) || !a16(y) || !a16(n_tok))
     return TWELL_ERR_INVALID_ARG;
   const int M = a->M, f = a->d_ff, tw = a->tile_w;
-  const TokLayout L = tok_layout(M, d_model, f, tw, cap_tok);
+  const TokLayout L = tok_layout(M, d_model, f, tw, a->ell_w, cap_tok);
   if (ws == nullptr || !a16(ws) || ws_bytes < L.total) return TWELL_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *base = static_cast<uint8_t *>(ws);

@@ -380,6 +380,40 @@ __device__ __forceinline__ void umma_commit_pair_mc(uint64_t *bar, uint16_t cta_
 }
 
 // ---------------------------------------------------------------------------
+// 2:4 structured-sparse MMA (tcgen05.mma.sp, kind::f16)
+//
+// A is stored compressed: per row, each group of 4 consecutive K elements keeps
+// 2 values (the shared-memory descriptor describes the compressed matrix like a
+// dense K-major one with K/2 columns).  The metadata lives in TMEM, one 32-bit
+// column per MMA of K = 32 (logical): the 4-bit code of a group holds the two
+// kept positions i0 < i1 as i0 | i1 << 2.  Row m and logical k of one MMA sit at
+//   lane 16 * (m / 16) + (m % 8) + 8 * ((k / 16) % 2),
+//   bit  (k % 16) + 16 * ((m / 8) % 2)
+// (checked on a B200 against an identity B operand).  The metadata address is
+// an even column; its low bit goes to the instruction descriptor's selector
+// field (bits 0..1).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void umma_sp_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                  uint32_t idesc, uint32_t meta_col_addr, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, {%6, %7, %8, %9, %10, %11, %12, %13}, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc | (meta_col_addr & 1u)), "r"(accumulate),
+      "r"(meta_col_addr & ~1u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+
+// 32 TMEM lanes x 4 consecutive 32-bit columns from registers: thread i writes
+// lane (base lane + i).  Complete with tmem_st_wait() before signalling readers.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Descriptors
 // ---------------------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2), version 1.

@@ -198,6 +198,29 @@ cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_
 cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
                                int num_sms, bool pdl, cudaStream_t s);
 
+// Down path of a 128-token block (the block-path array the down kernels share).
+constexpr int kPathGather = 0;   // CUDA-core gather (k_spmm_gather)
+constexpr int kPathDense = 1;    // tensor cores on dense h tiles rebuilt from TwELL (k_spmm_mma)
+constexpr int kPathSparse = 2;   // 2:4 structured-sparse tensor cores + excess fix-up (k_spmm_sp)
+
+// 2:4 split of h for the structured-sparse down path: per token, the nonzeros
+// beyond the first two of an aligned group of 4 hidden units ("excess") are
+// listed (at most kSpXc per token; a 256-token group with more takes the dense
+// tensor-core path) and added on CUDA cores in the epilogue.
+constexpr int kSpXc = 32;
+bool sp_eligible(const TwellView &v, int d_model);
+// Workspace of the 2:4 path: per-token excess counts, lists and fp32 excess
+// products [M][d_model], the kept values [M][d_ff / 2] and their MMA position codes.
+size_t sp_ws_bytes(int M, int d_ff, int d_model);
+// k_sp_prep then k_sp_decide: the 2:4 operand, excess lists and products, and
+// per 256-token group its down path (gather below gather_below; 2:4 when
+// allow_sparse and no token exceeds kSpXc; else dense); also zeroes the dense
+// kernel's split counters (split_ctr may be NULL).  sp_ws: the sp_ws_bytes region.
+cudaError_t launch_sp_prep(const TwellView &v, const uint16_t *w_down, int d, void *sp_ws, float gather_below,
+                           bool allow_sparse, int32_t *blk_path, int32_t *split_ctr, bool pdl, cudaStream_t s);
+cudaError_t launch_spmm_sp(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y, const int32_t *blk_path,
+                           void *sp_ws, int num_sms, bool pdl, cudaStream_t s);
+
 // Density (nonzeros / (rows * d_ff)) of a 128-token block at or above which the
 // AUTO down-projection uses the tensor-core path.  Chosen from measurement.
 constexpr float kDownCrossoverDensity = 0.006f;

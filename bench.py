@@ -293,6 +293,8 @@ def run_ours(args):
         down_k = ("k_spmm_gather", "CUDA-core gather of W_down rows per nonzero")
     elif dec_down:
         down_k = ("k_spmm_dec", "decode batch: split-K clusters, DSMEM reduction")
+    elif args.mode == "sparse" and _sparse_ok(M, f, tw, E):
+        down_k = ("k_spmm_sp", "2:4 sparse tensor cores on tiles rebuilt from TwELL + excess on CUDA cores")
     else:
         down_k = ("k_spmm_mma", "tensor cores on h tiles rebuilt from TwELL")
     phases = {"up": phase(*up_k, up_flop, up_bytes, up_s),
@@ -329,7 +331,7 @@ def run_ours(args):
                            "useful_flop": rl["useful_flop"],
                            "unavoidable_bytes": rl["unavoidable_bytes"],
                            "touched_w_down_rows": touched, "peaks": peaks["source"]},
-        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d),
+        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d, _sparse_ok(M, f, tw, E)),
         "wall_s_timed_region": wall,
     }
     result["clocks"] = clk.summary()
@@ -389,19 +391,27 @@ def _decode_paths(M, f, tw, mode):
     return (M <= 256 and tw <= 128 and f % 128 == 0), (M <= 256 and mode != "gather")
 
 
-def _kernels_per_step(mode, dec_down=False, d_model=0):
-    # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter; spmm: auto adds
-    # k_block_path and launches both down kernels (each skips the token blocks
-    # the other owns); mma runs k_block_path too when the split schedule is
-    # possible (d_model > 256: it zeroes the arrival counters); the decode-size
-    # down path is one kernel
+def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False):
+    # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter.
+    # spmm in sparse mode, where the 2:4 path applies: k_sp_prep, k_sp_decide,
+    # k_spmm_sp and k_spmm_mma, each tensor kernel taking its own token groups.
+    # Otherwise auto: k_block_path, gather and k_spmm_mma; mma runs
+    # k_block_path too when the split schedule is possible (d_model > 256: it
+    # zeroes the arrival counters); the decode-size down path is one kernel.
     if dec_down:
         return 4 + 1
+    if sparse_ok and mode == "sparse":
+        return 4 + 4   # k_sp_prep, k_sp_decide, k_spmm_sp, k_spmm_mma
     if mode == "auto":
         return 4 + 3
-    if mode == "mma":
+    if mode in ("mma", "sparse"):
         return 4 + (2 if d_model > 256 else 1)
     return 4 + 1
+
+
+def _sparse_ok(M, f, tw, E):
+    """Shapes the library's 2:4 down path takes (its host-side eligibility rule)."""
+    return tw in (64, 128) and E % 8 == 0 and E <= 32 and f < 65536 and M > 256
 
 
 def _dense_baseline(x, wu, b, wd, args, flush, stream, dev, wg=None):
@@ -750,7 +760,7 @@ def main():
     ap.add_argument("--density", type=float, default=0.05)
     ap.add_argument("--M", type=int, default=4096)
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--mode", default="auto", choices=["auto", "gather", "mma"])
+    ap.add_argument("--mode", default="auto", choices=["auto", "gather", "mma", "sparse"])
     ap.add_argument("--workload", default="relu_15b", choices=WORKLOADS,
                     help="default: the 1.5B-scale layer the headline metric is quoted on")
     ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")

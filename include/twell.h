@@ -50,9 +50,18 @@ typedef enum {
 
 /* Down-projection path selection. */
 typedef enum {
-  TWELL_DOWN_AUTO = 0,   /* per 128-token block, by measured density crossover   */
+  TWELL_DOWN_AUTO = 0,   /* per 128-token block, by measured density crossover:
+                            GATHER below it, MMA at or above it                   */
   TWELL_DOWN_GATHER = 1, /* CUDA-core gather of W_down rows per packed nonzero    */
-  TWELL_DOWN_MMA = 2     /* tcgen05 tensor cores on h tiles rebuilt from TwELL    */
+  TWELL_DOWN_MMA = 2,    /* tcgen05 tensor cores on h tiles rebuilt from TwELL    */
+  TWELL_DOWN_SPARSE = 3  /* tcgen05 2:4 structured-sparse tensor cores: per group
+                            of 4 hidden units the first two nonzeros run on the
+                            sparse MMA, the rest are added on CUDA cores.  Taken
+                            per 256-token group when every token has at most 32
+                            such extra nonzeros (else MMA); tile_w 64 or 128,
+                            ell_w % 8 == 0 and <= 32, d_ff % 128 == 0, M > 256
+                            (other shapes run MMA).  Explicit only: on B200 it
+                            measured slower than MMA at every density.            */
 } twell_down_mode;
 
 /*

@@ -63,6 +63,9 @@ def test_traffic_lookup_follows_the_kernel_source(monkeypatch, tmp_path):
 def test_kernels_per_step():
     # reset, producer, backup scan, scatter + block pass, gather, tensor-core kernel
     assert bench._kernels_per_step("auto", False, 2048) == 7
+    # the 2:4 path (sparse mode only): prep, decision, 2:4 kernel, dense kernel
+    assert bench._kernels_per_step("auto", False, 2048, True) == 7
+    assert bench._kernels_per_step("sparse", False, 2048, True) == 8
     # + block pass (split counters) and the tensor-core kernel
     assert bench._kernels_per_step("mma", False, 2048) == 6
     assert bench._kernels_per_step("mma", False, 256) == 5
