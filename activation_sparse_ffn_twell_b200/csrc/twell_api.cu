@@ -339,6 +339,19 @@ CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+CUresult encode_tensor_map_kchunks(CUtensorMap *map, const void *base, uint64_t K, uint64_t rows,
+                                   uint32_t box_rows, uint32_t chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return CUDA_ERROR_NOT_INITIALIZED;
+  const cuuint64_t dims[3] = {64, rows, K / 64};
+  const cuuint64_t strides[2] = {K * 2, 128};   // a row; a 64-element chunk
+  const cuuint32_t box[3] = {64, box_rows, chunks};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 }  // namespace twell
 
 using namespace twell;

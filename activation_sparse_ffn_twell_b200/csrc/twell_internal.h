@@ -227,6 +227,14 @@ constexpr float kDownCrossoverDensity = 0.006f;
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved at run time so the
 // library loads on machines without a driver).
+// A K-major bf16 matrix [rows][K] (K % 64 == 0) as a 3-D tensor (64 elements,
+// rows, K / 64 chunks) with 128-byte swizzle: one box of box_rows x `chunks`
+// chunks lands in shared memory as `chunks` consecutive [box_rows][64] tiles,
+// the layout of as many separate 2-D boxes, in one TMA request (the TMA unit's
+// throughput is bounded per request as well as per byte).
+CUresult encode_tensor_map_kchunks(CUtensorMap *map, const void *base, uint64_t K, uint64_t rows,
+                                   uint32_t box_rows, uint32_t chunks);
+
 CUresult encode_tensor_map_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                               uint64_t row_pitch_bytes, uint32_t box_inner, uint32_t box_outer,
                               CUtensorMapSwizzle swizzle,
