@@ -289,10 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(&bfull[bst], B_BYTES);
               bfilled |= 1u << bst;
               uint8_t *dst = sB + bst * B_BYTES;
-#pragma unroll
-              for (int j = 0; j < B_BOXES; ++j)
-                tma_load_2d(dst + j * (kBlockK * 128), &tmap_wd, &bfull[bst], n_blk * kTN + h * kBN + j * 64,
-                            kb * kBlockK);
+              // the 256 columns as four 64-column chunks of one 3-D box
+              tma_load_3d(dst, &tmap_wd, &bfull[bst], 0, kb * kBlockK, (n_blk * kTN + h * kBN) / 64);
               if (++bst == kBStages) { bst = 0; bph ^= 1u; }
             }
           }
@@ -304,14 +302,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           filled |= 1u << stage;
           uint8_t *dst = sB + stage * B_BYTES;
           const int col_b = n_blk * kBN + static_cast<int>(rank) * (B_BOXES * 64);
+          if constexpr (PAIR) {
 #pragma unroll
-          for (int j = 0; j < B_BOXES; ++j) {
-            if constexpr (PAIR)
+            for (int j = 0; j < B_BOXES; ++j)
               tma_load_2d_pair(dst + j * (kBlockK * 128), &tmap_wd, map_to_cta(&full[stage], 0),
                                col_b + j * 64, kb * kBlockK);
-            else
-              tma_load_2d(dst + j * (kBlockK * 128), &tmap_wd, &full[stage], col_b + j * 64,
-                          kb * kBlockK);
+          } else {   // the tile's 256 columns as four 64-column chunks of one 3-D box
+            tma_load_3d(dst, &tmap_wd, &full[stage], 0, kb * kBlockK, col_b / 64);
           }
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
@@ -1098,6 +1095,11 @@ cudaError_t launch_spmm_mma(const TwellView &v, const uint16_t *w_down, int d, u
   }
   P.slot_ib = ib;
   const bool pair = down_uses_pair(v);
+  // single-CTA tiles read W_down through a 3-D view: a box of 64 K-rows x four
+  // 64-column chunks lands as the four [64][64] tiles of a 256-column stage in
+  // one TMA request (the unit's throughput is bounded per request)
+  if (!pair && encode_tensor_map_kchunks(&mw, w_down, d, v.f, kBlockK, 4) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   // 512-column tiles unless y has at most 256 columns (or CTA pairs are on):
   // measured 1.7x the throughput of 256-column tiles per y column, which
   // outweighs a worse-filled last wave of SMs

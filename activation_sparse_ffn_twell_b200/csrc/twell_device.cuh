@@ -162,6 +162,17 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
       : "memory");
 }
 
+// 3-D tile load (see encode_tensor_map_kchunks): several 128-byte-wide chunks
+// of a box in one request, completion counted on an mbarrier of this CTA.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *map, uint64_t *bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 // Asynchronous global -> shared copies (no register round trip), grouped per
 // thread; wait_group<N> waits until at most N of this thread's groups are pending.
 __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
