@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kDecUpThreads, 1)
 // ============================================================================ down
 struct DecDownParams {
   TwellView A;
+  const uint16_t *w_down;   // [d_ff][d] (row gathers of the touched-unit kernel)
   uint16_t *y;
   int d;
   int np;                 // MMA N: tokens rounded up to a multiple of 16
@@ -365,6 +366,132 @@ __device__ __forceinline__ void zero_row_128(uint8_t *rp, int row) {
 #pragma unroll
   for (int c = 0; c < 8; ++c)
     *reinterpret_cast<uint4 *>(rp + (((c + row) & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// ---- roles shared by the two split-K down kernels
+
+// W_down tiles by TMA (one thread): K steps [kb_lo, kb_hi), two 64-column boxes
+// per step (an M-major operand, 64-element groups 8 KB apart; columns past
+// d_model are outside the tensor and arrive as zeros).
+__device__ __forceinline__ void dec_down_tma(uint8_t *smem, int STAGE, int kStages, uint64_t *full,
+                                             uint64_t *empty, volatile int *abort_flag, const CUtensorMap *tmap_wd,
+                                             int col0, int kb_lo, int kb_hi, int32_t *status) {
+  int stage = 0; uint32_t phase = 0;
+  uint32_t filled = 0;
+  bool ok = true;
+  for (int kb = kb_lo; kb < kb_hi; ++kb) {
+    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+    mbar_arrive_expect_tx(&full[stage], kWBytes);
+    filled |= 1u << stage;
+    uint8_t *dst = smem + stage * STAGE;
+    tma_load_2d(dst, tmap_wd, &full[stage], col0, kb * kBlockK);
+    tma_load_2d(dst + 8192, tmap_wd, &full[stage], col0 + 64, kb * kBlockK);
+    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    raise_status(status, TWELL_ERR_TIMEOUT);
+    for (int i = 0; i < kStages; ++i) {   // let issued copies land
+      if (!((filled >> i) & 1u)) continue;
+      mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
+    }
+  }
+}
+
+// MMA issuer (one thread): n_steps K steps of the stage ring, A = W_down^T tile
+// (M-major: 16 hidden rows of 128 B per MMA, the two 64-column halves 8 KB
+// apart), B = h^T tile (K-major rows).  tm_full is committed also on abort, so
+// the epilogue never waits out its limit.
+__device__ __forceinline__ void dec_down_mma(uint8_t *smem, int STAGE, int kStages, uint64_t *full,
+                                             uint64_t *empty, uint64_t *tm_full, uint64_t *drain,
+                                             volatile int *abort_flag, uint32_t tmem_base, uint32_t idesc,
+                                             int n_steps, int32_t *status) {
+  int stage = 0; uint32_t phase = 0;
+  bool ok = true;
+  for (int i = 0; i < n_steps; ++i) {
+    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+    tc_fence_after();
+    const uint32_t w_addr = smem_u32(smem + stage * STAGE);
+    const uint32_t h_addr = w_addr + kWBytes;
+#pragma unroll
+    for (int k = 0; k < kBlockK / kUmmaK; ++k) {
+      const uint64_t adesc = smem_desc_sw128(w_addr + k * 2048, 8192, 1024);
+      const uint64_t bdesc = smem_desc_sw128(h_addr + k * 32, 16, 1024);
+      umma_bf16(tmem_base, adesc, bdesc, idesc, (i != 0 || k != 0) ? 1u : 0u);
+    }
+    umma_commit(&empty[stage]);
+    if (++stage == kStages) { stage = 0; phase ^= 1u; }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    raise_status(status, TWELL_ERR_TIMEOUT);
+  }
+  umma_commit(tm_full);
+  umma_commit(drain);
+  mbar_wait_bounded(drain, 0);
+}
+
+// Epilogue warps 2..5 (TMEM lane quarter = warp % 4): the CTA's fp32 partial
+// [M][128] into shared memory; zeros when the CTA had no K step.
+__device__ __forceinline__ void dec_down_partial(float *part, uint64_t *tm_full, volatile int *abort_flag,
+                                                 uint32_t tmem_base, int warp, int lane, int M, bool has_k,
+                                                 int32_t *status) {
+  const int q = warp & 3;
+  if (mbar_wait(tm_full, 0, abort_flag)) {
+    tc_fence_after();
+    const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+    const int c_local = 32 * q + lane;
+    const int nchunks = (M + 31) >> 5;
+    for (int c0 = 0; c0 < nchunks; ++c0) {
+      uint32_t v[32];
+      if (has_k) {
+        __syncwarp();
+        tmem_ld_32x32b_x32(trow + c0 * 32, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int tok = c0 * 32 + j;
+        if (tok < M) part[tok * kDecCols + c_local] = __uint_as_float(v[j]);
+      }
+    }
+  } else {
+    *abort_flag = 1;
+    raise_status(status, TWELL_ERR_TIMEOUT);
+  }
+}
+
+// Cluster reduction: CTA `rank` adds the partials of its share of the tokens
+// over the cluster's CTAs in rank order (distributed shared memory) and stores
+// y once, rounded to bf16.  Every thread of the cluster takes part.
+__device__ __forceinline__ void dec_down_reduce(const float *part, uint16_t *y, int M, int d, int split,
+                                                uint32_t rank, int col0) {
+  __syncwarp();
+  cluster_sync();
+  const int per = (M + split - 1) / split;
+  const int tok0 = static_cast<int>(rank) * per;
+  const int ntok = max(0, min(M, tok0 + per) - tok0);
+  for (int i = threadIdx.x; i < ntok * (kDecCols / 4); i += blockDim.x) {
+    const int tok = tok0 + i / (kDecCols / 4);
+    const int c4 = (i % (kDecCols / 4)) * 4;
+    const int gc = col0 + c4;
+    if (gc >= d) continue;
+    const float *src = part + tok * kDecCols + c4;
+    float4 acc = ld_shared_cluster_f4(map_to_cta(src, 0));
+    for (int r = 1; r < split; ++r) {
+      const float4 v = ld_shared_cluster_f4(map_to_cta(src, static_cast<uint32_t>(r)));
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<uint2 *>(y + static_cast<size_t>(tok) * d + gc) =
+        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();   // no CTA leaves while a peer still reads its partial
+  tc_fence_after();
 }
 
 // EV: ell_w / 8 on the fast builder path (ell_w % 8 == 0, tile_w >= 64), else 0.
@@ -414,81 +541,16 @@ __global__ void __launch_bounds__(kDecDownThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA: W_down tiles
-    if (lane == 0) {
-      int stage = 0; uint32_t phase = 0;
-      uint32_t filled = 0;
-      bool ok = true;
-      for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[stage], kWBytes);
-        filled |= 1u << stage;
-        uint8_t *dst = smem + stage * STAGE;
-        // two 64-column boxes: an M-major operand, 64-element groups 8 KB apart
-        // (columns past d_model are outside the tensor and arrive as zeros)
-        tma_load_2d(dst, &tmap_wd, &full[stage], col0, kb * kBlockK);
-        tma_load_2d(dst + 8192, &tmap_wd, &full[stage], col0 + 64, kb * kBlockK);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        raise_status(A.status, TWELL_ERR_TIMEOUT);
-        for (int i = 0; i < kStages; ++i) {
-          if (!((filled >> i) & 1u)) continue;
-          mbar_wait_bounded(&full[i], (i < stage) ? phase : (phase ^ 1u));
-        }
-      }
-    }
+    if (lane == 0)
+      dec_down_tma(smem, STAGE, kStages, full, empty, abort_flag, &tmap_wd, col0, kb_lo, kb_hi, A.status);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0; uint32_t phase = 0;
-      bool ok = true;
-      for (int kb = kb_lo; kb < kb_hi; ++kb) {
-        if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t w_addr = smem_u32(smem + stage * STAGE);
-        const uint32_t h_addr = w_addr + kWBytes;
-#pragma unroll
-        for (int k = 0; k < kBlockK / kUmmaK; ++k) {
-          // A (W_down^T): 16 hidden rows of 128 B per step; B (h^T): K-major rows
-          const uint64_t adesc = smem_desc_sw128(w_addr + k * 2048, 8192, 1024);
-          const uint64_t bdesc = smem_desc_sw128(h_addr + k * 32, 16, 1024);
-          umma_bf16(tmem_base, adesc, bdesc, P.idesc, (kb != kb_lo || k != 0) ? 1u : 0u);
-        }
-        umma_commit(&empty[stage]);
-        if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        raise_status(A.status, TWELL_ERR_TIMEOUT);
-      }
-      umma_commit(tm_full);   // also issued on abort: the epilogue must not wait out its limit
-      umma_commit(drain);
-      mbar_wait_bounded(drain, 0);
-    }
+    if (lane == 0)
+      dec_down_mma(smem, STAGE, kStages, full, empty, tm_full, drain, abort_flag, tmem_base, P.idesc,
+                   kb_hi - kb_lo, A.status);
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue: TMEM -> partial
-    const int q = warp & 3;
-    if (mbar_wait(tm_full, 0, abort_flag)) {
-      tc_fence_after();
-      const uint32_t trow = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-      const int c_local = 32 * q + lane;
-      const int nchunks = (A.M + 31) >> 5;
-      for (int c0 = 0; c0 < nchunks; ++c0) {
-        uint32_t v[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(trow + c0 * 32, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tok = c0 * 32 + j;
-          if (tok < A.M) part[tok * kDecCols + c_local] = __uint_as_float(v[j]);
-        }
-      }
-    } else {
-      *abort_flag = 1;
-      raise_status(A.status, TWELL_ERR_TIMEOUT);
-    }
+    dec_down_partial(part, tm_full, abort_flag, tmem_base, warp, lane, A.M, true, A.status);
   } else {
     // ------------------------------------------------------------ builders: h^T tiles
     // thread = token row of the operand; row i of a stage holds hidden columns
@@ -626,32 +688,454 @@ __global__ void __launch_bounds__(kDecDownThreads, 1)
     }
   }
 
-  // ---- cluster reduction: CTA `rank` adds the partials of its share of tokens
-  __syncwarp();
-  cluster_sync();
-  {
-    const int per = (A.M + P.split - 1) / P.split;
-    const int tok0 = static_cast<int>(rank) * per;
-    const int ntok = max(0, min(A.M, tok0 + per) - tok0);
-    for (int i = threadIdx.x; i < ntok * (kDecCols / 4); i += blockDim.x) {
-      const int tok = tok0 + i / (kDecCols / 4);
-      const int c4 = (i % (kDecCols / 4)) * 4;
-      const int gc = col0 + c4;
-      if (gc >= P.d) continue;
-      const float *src = part + tok * kDecCols + c4;
-      float4 acc = ld_shared_cluster_f4(map_to_cta(src, 0));
-      for (int r = 1; r < P.split; ++r) {
-        const float4 v = ld_shared_cluster_f4(map_to_cta(src, static_cast<uint32_t>(r)));
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      *reinterpret_cast<uint2 *>(P.y + static_cast<size_t>(tok) * P.d + gc) =
-          make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  dec_down_reduce(part, P.y, A.M, P.d, P.split, rank, col0);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
+// ============================================================================ touched units
+// Bit u of the bitmap is set when some token has h[token][u] != 0: a TwELL slot
+// of a pair within ell_w, or a nonzero in the dense backup segment of an
+// overflowing pair.  A CTA owns kTouchUnits consecutive hidden units (whole
+// tiles, tile_w <= 256) and writes its bitmap words once, so no zeroing pass
+// is needed.
+constexpr int kTouchUnits = 256;
+
+__global__ void __launch_bounds__(256) k_dec_touch(const TwellView A, uint32_t *bitmap) {
+  __shared__ uint32_t words[kTouchUnits / 32];
+  griddep_launch_dependents();
+  if (threadIdx.x < kTouchUnits / 32) words[threadIdx.x] = 0u;
+  __syncthreads();
+  griddep_wait();
+  const int u0 = blockIdx.x * kTouchUnits;
+  const int t0 = u0 / A.tw;
+  const int t1 = min(A.T, t0 + kTouchUnits / A.tw);
+  const int nt = t1 - t0;
+  // pairs within ell_w: their slots
+  for (int i = threadIdx.x; i < A.M * nt; i += blockDim.x) {
+    const int tok = i / nt, t = t0 + i % nt;
+    const size_t pair = static_cast<size_t>(tok) * A.T + t;
+    const int n = __ldg(A.nnz + pair);
+    if (n > A.E) continue;
+    const int ub = t * A.tw - u0;                     // CTA-local unit of in-tile index 0
+    const uint8_t *si = A.idx + pair * A.E;
+    for (int e = 0; e < n; ++e) {
+      const int u = ub + __ldg(si + e);
+      if (u < kTouchUnits) atomicOr(&words[u >> 5], 1u << (u & 31));   // in-tile index < tile_w
     }
   }
+  // overflowing pairs: the nonzeros of their backup segments (the list is
+  // scanned by every CTA; each takes the segments of its own tiles)
+  const int n_ovf = min(*A.n_ovf, A.cap);
+  const int vec = A.tw / 8;                           // 16-byte pieces per segment
+  for (int i = threadIdx.x; i < n_ovf * vec; i += blockDim.x) {
+    const int k = i / vec, c8 = (i % vec) * 8;
+    const int t = __ldg(A.ovf_pos + k) % A.T;
+    if (t < t0 || t >= t1) continue;
+    const uint4 q = __ldg(reinterpret_cast<const uint4 *>(A.ovf_dense + static_cast<size_t>(k) * A.tw + c8));
+    const uint32_t h[4] = {q.x, q.y, q.z, q.w};
+    uint32_t m = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if ((h[j >> 1] >> (16 * (j & 1))) & 0x7FFFu) m |= 1u << j;
+    if (m != 0u) {
+      const int u = t * A.tw - u0 + c8;               // 8 units inside one 32-unit word
+      atomicOr(&words[u >> 5], m << (u & 31));
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < kTouchUnits / 32) {
+    const int w = u0 / 32 + static_cast<int>(threadIdx.x);
+    if (w * 32 < A.f) bitmap[w] = words[threadIdx.x];
+  }
+}
+
+// Gather mode when at most kGatherNum / kGatherDen of the hidden units are
+// touched; above that every W_down row is streamed by TMA as in k_spmm_dec.
+constexpr int kGatherNum = 3, kGatherDen = 4;
+constexpr int kGatherLag = 4;          // stages a gather thread keeps in flight before signalling one
+constexpr size_t kDecTablesOff = 512;  // the lookup tables follow the barrier block
+
+// Split-K down-projection over the touched hidden units only.  Every CTA reads
+// the bitmap, scans it (position of each touched unit in the compacted K) and
+// lists the units of its share of the compacted K steps.  A K step then holds
+// the W_down rows of 64 touched units (gathered by warps 2..5 with 16-byte
+// asynchronous copies into the same swizzled operand layout the TMA writes)
+// and the h^T columns of the same units (builders map a slot's unit to its
+// compacted column).  Untouched rows multiply h columns that are zero for
+// every token of the batch, so y is unchanged.
+template <int EV>
+__global__ void __launch_bounds__(kDecDownThreads, 1)
+    k_spmm_dec_touched(const __grid_constant__ CUtensorMap tmap_wd, const DecDownParams P,
+                       const uint32_t *__restrict__ bitmap) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  const int kStages = P.stages;
+  const int STAGE = kWBytes + P.np * 128;                 // [W_down tile][h^T tile]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kStages * STAGE);
+  uint64_t *full = bars;
+  uint64_t *empty = bars + kDecMaxStages;
+  uint64_t *tm_full = bars + 2 * kDecMaxStages;
+  uint64_t *drain = tm_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tm_full + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  int *scan_s = reinterpret_cast<int *>(bars + 32);        // per-warp totals of the scan
+  const TwellView &A = P.A;
+  const int W = A.f >> 5;                                  // bitmap words (d_ff % 32 == 0)
+  uint32_t *bm_s = reinterpret_cast<uint32_t *>(smem + kStages * STAGE + kDecTablesOff);   // [W + 1]
+  int *pre_s = reinterpret_cast<int *>(bm_s + W + 1);      // [W + 1]: touched units before word w
+  uint16_t *u_s = reinterpret_cast<uint16_t *>(pre_s + W + 1);   // units of this CTA's share
+  float *part = reinterpret_cast<float *>(smem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const uint32_t rank = cluster_ctarank();
+  const int col0 = static_cast<int>(cluster_id_x()) * kDecCols;
+
+  // ---- touched-unit tables (every role needs them; the bitmap comes from the
+  // previous kernel)
+  griddep_wait();
+  const int per = (W + nth - 1) / nth;
+  const int w0 = min(W, tid * per), w1 = min(W, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t b = __ldg(bitmap + w);
+    bm_s[w] = b;
+    cnt += __popc(b);
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) scan_s[warp] = incl;
+  __syncthreads();
+  int run = 0, touched = 0;
+  for (int i = 0; i < (nth >> 5); ++i) {
+    const int v = scan_s[i];
+    if (i < warp) run += v;
+    touched += v;
+  }
+  run += incl - cnt;
+  const bool gather = static_cast<long long>(touched) * kGatherDen <= static_cast<long long>(A.f) * kGatherNum;
+  for (int w = w0; w < w1; ++w) {
+    if (gather) {
+      pre_s[w] = run;
+      run += __popc(bm_s[w]);
+    } else {                                               // every unit in place
+      bm_s[w] = 0xFFFFFFFFu;
+      pre_s[w] = 32 * w;
+    }
+  }
+  const int Kc = gather ? touched : A.f;                   // compacted K
+  if (tid == 0) { bm_s[W] = 0u; pre_s[W] = Kc; }
+  __syncthreads();
+  const int nsteps = (Kc + kBlockK - 1) / kBlockK;
+  const int kb_lo = static_cast<int>((static_cast<long long>(rank) * nsteps) / P.split);
+  const int kb_hi = static_cast<int>((static_cast<long long>(rank + 1) * nsteps) / P.split);
+  const int p_lo = kb_lo * kBlockK, p_hi = min(kb_hi * kBlockK, Kc);
+  const bool has_k = kb_hi > kb_lo;
+  if (gather) {
+    for (int w = tid; w < W; w += nth) {
+      int p = pre_s[w];
+      if (pre_s[w + 1] <= p_lo || p >= p_hi) continue;
+      uint32_t b = bm_s[w];
+      while (b != 0u) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1u;
+        if (p >= p_lo && p < p_hi) u_s[p - p_lo] = static_cast<uint16_t>(32 * w + bit);
+        ++p;
+      }
+    }
+  }
+  // unit of compacted column p (p_lo <= p < p_hi); compacted column of touched unit u
+  auto unit_at = [&](int p) -> int { return gather ? static_cast<int>(u_s[p - p_lo]) : p; };
+  auto pos_of = [&](int u) -> int {
+    const int w = u >> 5;
+    return pre_s[w] + __popc(bm_s[w] & ((1u << (u & 31)) - 1u));
+  };
+  auto is_touched = [&](int u) -> bool { return (bm_s[u >> 5] >> (u & 31)) & 1u; };
+
+  // builder warps per step: enough for the operand's np rows (a power of two)
+  const int wpg = P.np <= 32 ? 1 : P.np <= 64 ? 2 : P.np <= 128 ? 4 : 8;
+  if (tid == 0) {
+    // full: the W tile (one TMA arrival with its bytes, or the 4 gather warps)
+    // and the wpg builder warps of the step
+    for (int i = 0; i < kStages; ++i) { mbar_init(&full[i], (gather ? 4 : 1) + wpg); mbar_init(&empty[i], 1); }
+    mbar_init(tm_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (!gather) tma_prefetch_desc(&tmap_wd);
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, P.tmem_cols); tmem_relinquish(); }
   tc_fence_before();
-  __syncwarp();
-  cluster_sync();   // no CTA leaves while a peer still reads its partial
+  __syncthreads();
   tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (!gather && lane == 0)
+      dec_down_tma(smem, STAGE, kStages, full, empty, abort_flag, &tmap_wd, col0, kb_lo, kb_hi, A.status);
+  } else if (warp == 1) {
+    if (lane == 0)
+      dec_down_mma(smem, STAGE, kStages, full, empty, tm_full, drain, abort_flag, tmem_base, P.idesc,
+                   kb_hi - kb_lo, A.status);
+  } else if (warp < 6) {
+    if (gather) {
+      // ---------------------------------------------------------- W_down row gather
+      // thread: 16-byte chunk c16 of the 256-byte row piece [col0, col0 + 128),
+      // rows r0 + 8 i of the K step; chunk c16 lands in 64-column half c16 / 8
+      // at the 128-byte swizzled place of its row
+      const int pt = tid - 64;
+      const int c16 = pt & 15, r0 = pt >> 4;
+      const int gcol = col0 + c16 * 8;
+      const bool col_ok = gcol < P.d;
+      const uint32_t chunk = static_cast<uint32_t>(c16 & 7);
+      const uint32_t half = static_cast<uint32_t>(c16 >> 3) * 8192u;
+      int stage = 0; uint32_t phase = 0;
+      int issued = 0, sig = 0;                             // groups issued; next stage to signal
+      bool ok = true;
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t *base = smem + stage * STAGE;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int row = r0 + 8 * i;
+          const int p = kb * kBlockK + row;
+          const bool live = col_ok && p < p_hi;
+          const uint16_t *src = live ? P.w_down + static_cast<size_t>(u_s[p - p_lo]) * P.d + gcol : P.w_down;
+          const uint32_t off = half + static_cast<uint32_t>(row) * 128u +
+                               ((chunk ^ static_cast<uint32_t>(row & 7)) << 4);
+          cp_async_16_zfill(base + off, src, live ? 16u : 0u);
+        }
+        cp_async_commit();
+        if (++issued > kGatherLag) {
+          cp_async_wait<kGatherLag>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[sig]);
+          if (++sig == kStages) sig = 0;
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      for (int i = min(issued, kGatherLag); i > 0; --i) {
+        if (lane == 0) mbar_arrive(&full[sig]);
+        if (++sig == kStages) sig = 0;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_status(A.status, TWELL_ERR_TIMEOUT);
+      }
+    }
+    dec_down_partial(part, tm_full, abort_flag, tmem_base, warp, lane, A.M, has_k, A.status);
+  } else {
+    // ------------------------------------------------------------ builders: h^T tiles
+    // thread = token row; row i of a stage holds compacted columns
+    // [64 kb, 64 kb + 64) of token i, 128-byte swizzled.  A step covers the
+    // units [unit_at(64 kb), unit_at(64 kb + 63)], i.e. the tiles between them.
+    // The 8 builder warps form 8 / wpg groups of wpg warps (enough warps for
+    // the operand's rows); group g builds the steps kb_lo + g + i * groups, so
+    // with a few tokens several steps are built at once and the latency of
+    // their TwELL record loads overlaps.
+    const int bw = warp - 6;
+    const int groups = 8 / wpg, grp = bw / wpg;
+    const int row = (bw % wpg) * 32 + lane;
+    const bool live = row < A.M;
+    const bool in_op = row < P.np;                           // the operand has np rows
+    const int tw = A.tw, E = A.E, Tn = A.T;
+    const int lg_tw = 31 - __clz(tw);
+    const int n_ovf = min(*A.n_ovf, A.cap);
+    const uint32_t row_swz = static_cast<uint32_t>(row & 7);
+    const size_t pair0 = static_cast<size_t>(live ? row : 0) * Tn;
+    auto put = [&](uint8_t *rp, int col, uint32_t v) {
+      const uint32_t c = static_cast<uint32_t>(col);
+      *reinterpret_cast<uint16_t *>(rp + ((((c >> 3) ^ row_swz) << 4) + ((c & 7u) << 1))) = static_cast<uint16_t>(v);
+    };
+    // the dense backup segment k of tile t: its units in this step, eight
+    // loads in flight at a time
+    auto put_backup = [&](uint8_t *rp, int t, int k, int p0) {
+      const int q_lo = max(p0, pos_of(t << lg_tw));
+      const int q_hi = min(min(p0 + kBlockK, p_hi), pos_of((t + 1) << lg_tw));
+      const uint16_t *src = A.ovf_dense + static_cast<size_t>(k) * tw - (t << lg_tw);
+      for (int q = q_lo; q < q_hi; q += 8) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = (q + j < q_hi) ? __ldg(src + unit_at(q + j)) : 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (q + j < q_hi) put(rp, q + j - p0, v[j]);
+      }
+    };
+    // this row's backup entries, walked in tile order (a group's tiles only grow)
+    int walk = n_ovf;
+    if (live && kb_lo + grp < kb_hi)
+      walk = ovf_lower_bound(A.ovf_pos, n_ovf, static_cast<int>(pair0) + (unit_at((kb_lo + grp) * kBlockK) >> lg_tw));
+    auto find_ovf = [&](int t) -> int {
+      while (walk < n_ovf && __ldg(A.ovf_pos + walk) < static_cast<int>(pair0) + t) ++walk;
+      return (walk < n_ovf && __ldg(A.ovf_pos + walk) == static_cast<int>(pair0) + t) ? walk : -1;
+    };
+    // the records of this row's tiles in the CTA's share, asked of L2 up front
+    // (group 0 only: the groups share the rows)
+    if (live && has_k && grp == 0) {
+      const size_t ta = static_cast<size_t>(unit_at(p_lo) >> lg_tw);
+      const size_t nt = static_cast<size_t>(unit_at(p_hi - 1) >> lg_tw) - ta + 1;
+      prefetch_l2_range(A.vals + (pair0 + ta) * E, nt * E * 2);
+      prefetch_l2_range(A.idx + (pair0 + ta) * E, nt * E);
+      prefetch_l2_range(A.nnz + pair0 + ta, nt * 2);
+    }
+    bool ok = true;
+    if constexpr (EV > 0) {
+      // A tile's record (values, indices, count) is loaded into registers; the
+      // first tiles of the group's next step are loaded while this step is
+      // built.  A warp walks the tiles together: lane j holds bitmap word j of
+      // the tile and the touched units of the tile before it, and a slot's
+      // compacted column comes from two shuffles (no per-slot table reads).
+      constexpr int EF = 8 * EV;
+      constexpr int NPF = EV == 1 ? 2 : 1;                  // tiles of a step loaded ahead
+      struct Rec { uint4 v[EV]; uint2 ix[EV]; int n; };
+      auto fetch = [&](int t, Rec &r) {
+        if (live && t < Tn) {
+          const uint4 *gv = reinterpret_cast<const uint4 *>(A.vals + (pair0 + t) * EF);
+          const uint2 *gi = reinterpret_cast<const uint2 *>(A.idx + (pair0 + t) * EF);
+#pragma unroll
+          for (int g = 0; g < EV; ++g) { r.v[g] = __ldg(gv + g); r.ix[g] = __ldg(gi + g); }
+          r.n = static_cast<int>(__ldg(A.nnz + pair0 + t));
+        } else {
+          r.n = 0;
+        }
+      };
+      const int nw = tw >> 5;
+      uint32_t t_word = 0u;
+      int t_before = 0, t_pos = 0;
+      auto tile_map = [&](int t) {                           // warp-uniform
+        const int wb = t << (lg_tw - 5);
+        t_word = lane < nw ? bm_s[wb + lane] : 0u;
+        int c = __popc(t_word);
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, c, o);
+          if (lane >= o) c += v;
+        }
+        t_before = c - __popc(t_word);
+        t_pos = pre_s[wb];
+      };
+      auto emit = [&](uint8_t *rp, const Rec &r, int t, int ulo, int uhi, int p0) {
+        const bool slots = r.n > 0 && r.n <= EF;
+        const int u_t = t << lg_tw;
+#pragma unroll
+        for (int g = 0; g < EV; ++g) {
+          const uint32_t vw[4] = {r.v[g].x, r.v[g].y, r.v[g].z, r.v[g].w};
+          const uint32_t iw[2] = {r.ix[g].x, r.ix[g].y};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int ix = static_cast<int>((iw[e >> 2] >> (8 * (e & 3))) & 0xFFu);
+            const uint32_t wj = __shfl_sync(0xFFFFFFFFu, t_word, ix >> 5);
+            const int cj = __shfl_sync(0xFFFFFFFFu, t_before, ix >> 5);
+            const int u = u_t + ix;
+            if (slots && 8 * g + e < r.n && ix < tw && u >= ulo && u <= uhi && ((wj >> (ix & 31)) & 1u))
+              put(rp, t_pos + cj + __popc(wj & ((1u << (ix & 31)) - 1u)) - p0, vw[e >> 1] >> (16 * (e & 1)));
+          }
+        }
+        if (r.n > EF) {
+          const int k = find_ovf(t);
+          if (k >= 0) put_backup(rp, t, k, p0);
+        }
+      };
+      Rec cur[NPF], nxt[NPF];
+      int nxt_t0 = -1;
+      for (int kb = kb_lo + grp; kb < kb_hi; kb += groups) {
+        const int i = kb - kb_lo;
+        const int stage = i % kStages;
+        const uint32_t par = static_cast<uint32_t>((i / kStages) & 1) ^ 1u;
+        const int p0 = kb * kBlockK;
+        const int ulo = unit_at(p0), uhi = unit_at(min(p0 + kBlockK, p_hi) - 1);
+        const int t_lo = ulo >> lg_tw, t_hi = uhi >> lg_tw;
+        if (nxt_t0 == t_lo) {
+#pragma unroll
+          for (int j = 0; j < NPF; ++j) cur[j] = nxt[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < NPF; ++j) fetch(t_lo + j, cur[j]);
+        }
+        nxt_t0 = -1;
+        if (kb + groups < kb_hi) {
+          nxt_t0 = unit_at((kb + groups) * kBlockK) >> lg_tw;
+#pragma unroll
+          for (int j = 0; j < NPF; ++j) fetch(nxt_t0 + j, nxt[j]);
+        }
+        // the lanes leave together (the shuffles need the whole warp)
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[stage], par, abort_flag))) { ok = false; break; }
+        uint8_t *rp = smem + stage * STAGE + kWBytes + row * 128;
+        if (in_op) zero_row_128(rp, row);
+        for (int t = t_lo; t <= t_hi; ++t) {                 // warp-uniform
+          tile_map(t);
+          const int j = t - t_lo;
+          if (j < NPF) {
+#pragma unroll
+            for (int jj = 0; jj < NPF; ++jj)
+              if (jj == j) emit(rp, cur[jj], t, ulo, uhi, p0);
+          } else {
+            Rec r;
+            fetch(t, r);
+            emit(rp, r, t, ulo, uhi, p0);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+      }
+    } else {
+      // any ell_w / tile_w: the row's counts and slots are read per tile
+      for (int kb = kb_lo + grp; kb < kb_hi; kb += groups) {
+        const int i = kb - kb_lo;
+        const int stage = i % kStages;
+        const uint32_t par = static_cast<uint32_t>((i / kStages) & 1) ^ 1u;
+        const int p0 = kb * kBlockK;
+        const int ulo = unit_at(p0), uhi = unit_at(min(p0 + kBlockK, p_hi) - 1);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(&empty[stage], par, abort_flag))) { ok = false; break; }
+        if (in_op) {
+          uint8_t *rp = smem + stage * STAGE + kWBytes + row * 128;
+          zero_row_128(rp, row);
+          if (live) {
+            for (int t = ulo >> lg_tw; t <= (uhi >> lg_tw); ++t) {
+              const size_t pair = pair0 + t;
+              const int n = __ldg(A.nnz + pair);
+              if (n == 0) continue;
+              if (n <= E) {
+                const uint16_t *sv = A.vals + pair * E;
+                const uint8_t *si = A.idx + pair * E;
+                for (int e = 0; e < n; ++e) {
+                  const int u = (t << lg_tw) + __ldg(si + e);
+                  if (u >= ulo && u <= uhi && is_touched(u)) put(rp, pos_of(u) - p0, __ldg(sv + e));
+                }
+              } else {
+                const int k = find_ovf(t);
+                if (k >= 0) put_backup(rp, t, k, p0);
+              }
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      raise_status(A.status, TWELL_ERR_TIMEOUT);
+    }
+  }
+
+  dec_down_reduce(part, P.y, A.M, P.d, P.split, rank, col0);
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem_base, P.tmem_cols);
@@ -741,6 +1225,24 @@ bool decode_enabled() {
   return v == 1;
 }
 
+// Batches that take the touched-unit down kernel: TWELL_DECODE_TOUCHED=0 never,
+// =all every decode-size batch, unset up to kDecTouchedMaxTokens tokens.  On
+// B200 at 4096 -> 16384 and 2 % density it took 36-38 us against 47.6 us for
+// the streaming kernel at 32 tokens (about half of W_down's rows touched), but
+// 62-72 us against 53 us at 64 tokens (73 % touched), where its builders (one
+// group of two warps per K step, four steps in flight) fall behind; the
+// streaming kernel can also start reading W_down before the up-projection ends.
+constexpr int kDecTouchedMaxTokens = 32;
+
+bool dec_touched_for(int M) {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("TWELL_DECODE_TOUCHED");
+    v = (e == nullptr) ? 1 : (e[0] == '0') ? 0 : (e[0] == 'a') ? 2 : 1;
+  }
+  return v == 2 || (v == 1 && M <= kDecTouchedMaxTokens);
+}
+
 }  // namespace
 
 bool decode_up_eligible(int M, int d_ff, int tile_w) {
@@ -760,47 +1262,45 @@ cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_
   }
 }
 
-cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y, int num_sms,
-                               bool pdl, cudaStream_t s) {
+cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
+                               uint32_t *touch_ws, int num_sms, bool pdl, cudaStream_t s) {
   if (v.M == 0) return cudaSuccess;
   DecDownParams P;
   P.A = v;
+  P.w_down = w_down;
   P.y = y;
   P.d = d;
   P.np = round_tokens(v.M);
   P.num_kb = (v.f + kBlockK - 1) / kBlockK;
   P.tmem_cols = tmem_cols_for(P.np);
   P.idesc = idesc_bf16_f32(kDecCols, P.np, 1, 0);
-  const size_t stage = static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
-  const size_t extra = 1024 + 512;
-  int stages = static_cast<int>((kDecSmemBudget - extra) / stage);
-  if (stages > kDecMaxStages) stages = kDecMaxStages;
-  // the partial [np][128] fp32 reuses the stage buffers
-  if (stages < 2 || static_cast<size_t>(stages) * stage < static_cast<size_t>(P.np) * kDecCols * 4)
-    return cudaErrorInvalidValue;
-  P.stages = stages;
-  const size_t smem = extra + stages * stage;
+  bool touched = touch_ws != nullptr && dec_touched_for(v.M) && v.f <= 65536;
   const int ev = (v.E % 8 == 0 && v.E <= 64 && v.tw >= 64) ? v.E / 8 : 0;
   void (*kern)(const CUtensorMap, const DecDownParams) = nullptr;
+  void (*kern_t)(const CUtensorMap, const DecDownParams, const uint32_t *) = nullptr;
   switch (ev) {
-    case 1: kern = k_spmm_dec<1>; break;
-    case 2: kern = k_spmm_dec<2>; break;
-    case 3: kern = k_spmm_dec<3>; break;
-    case 4: kern = k_spmm_dec<4>; break;
-    case 5: kern = k_spmm_dec<5>; break;
-    case 6: kern = k_spmm_dec<6>; break;
-    case 7: kern = k_spmm_dec<7>; break;
-    case 8: kern = k_spmm_dec<8>; break;
-    default: kern = k_spmm_dec<0>; break;
+    case 1: kern = k_spmm_dec<1>; kern_t = k_spmm_dec_touched<1>; break;
+    case 2: kern = k_spmm_dec<2>; kern_t = k_spmm_dec_touched<2>; break;
+    case 3: kern = k_spmm_dec<3>; kern_t = k_spmm_dec_touched<3>; break;
+    case 4: kern = k_spmm_dec<4>; kern_t = k_spmm_dec_touched<4>; break;
+    case 5: kern = k_spmm_dec<5>; kern_t = k_spmm_dec_touched<5>; break;
+    case 6: kern = k_spmm_dec<6>; kern_t = k_spmm_dec_touched<6>; break;
+    case 7: kern = k_spmm_dec<7>; kern_t = k_spmm_dec_touched<7>; break;
+    case 8: kern = k_spmm_dec<8>; kern_t = k_spmm_dec_touched<8>; break;
+    default: kern = k_spmm_dec<0>; kern_t = k_spmm_dec_touched<0>; break;
   }
   // the attribute is the full budget, so the occupancy query below sees the
   // same limit at every token count
   cudaError_t e = cudaFuncSetAttribute(k_spmm_dec<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kDecSmemBudget));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kDecSmemBudget));
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDecSmemBudget));
   if (e != cudaSuccess) return e;
+  if (touched) {
+    e = cudaFuncSetAttribute(kern_t, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kDecSmemBudget));
+    if (e != cudaSuccess) return e;
+  }
   // Split K so that the clusters fill the GPU: the cost of a split is the
   // number of waves of clusters times the K steps per CTA.
   const int n_slices = (d + kDecCols - 1) / kDecCols;
@@ -815,12 +1315,46 @@ cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d
     if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = split; }
   }
   P.split = best;
+  // shared memory: stage ring, barrier block, and (touched-unit kernel) the
+  // bitmap, its prefix and the unit list of one CTA's share of K
+  const size_t stage = static_cast<size_t>(kWBytes) + static_cast<size_t>(P.np) * 128;
+  auto ring = [&](size_t tables) -> int {
+    const size_t extra = 1024 + kDecTablesOff + ((tables + 15) & ~static_cast<size_t>(15));
+    if (extra >= kDecSmemBudget) return 0;
+    const size_t n = (kDecSmemBudget - extra) / stage;
+    return static_cast<int>(n < static_cast<size_t>(kDecMaxStages) ? n : static_cast<size_t>(kDecMaxStages));
+  };
+  size_t tables = 0;
+  if (touched) {
+    const size_t W = static_cast<size_t>(v.f / 32);
+    const size_t share = static_cast<size_t>((P.num_kb + best - 1) / best) * kBlockK;
+    tables = 8 * (W + 1) + 2 * share;
+    // the gather keeps kGatherLag stages in flight before it signals one: with
+    // a shorter ring (large batches) every row is streamed instead
+    if (ring(tables) <= kGatherLag) { touched = false; tables = 0; }
+  }
+  const size_t extra = 1024 + kDecTablesOff + ((tables + 15) & ~static_cast<size_t>(15));
+  const int stages = ring(tables);
+  // the partial [np][128] fp32 reuses the stage buffers
+  if (stages < 2 || static_cast<size_t>(stages) * stage < static_cast<size_t>(P.np) * kDecCols * 4)
+    return cudaErrorInvalidValue;
+  P.stages = stages;
+  const size_t smem = extra + stages * stage;
   CUtensorMap mw;
   if (encode_tensor_map_2d(&mw, w_down, d, v.f, static_cast<uint64_t>(d) * 2, 64, kBlockK,
                            CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  return launch_k(kern, dim3(n_slices * best), dim3(kDecDownThreads), smem, s, pdl,
-                  static_cast<unsigned>(best), mw, P);
+  if (!touched)
+    return launch_k(kern, dim3(n_slices * best), dim3(kDecDownThreads), smem, s, pdl,
+                    static_cast<unsigned>(best), mw, P);
+  e = launch_k(k_dec_touch, dim3((v.f + kTouchUnits - 1) / kTouchUnits), dim3(256), 0, s, pdl, 1u, v, touch_ws);
+  if (e != cudaSuccess) return e;
+  return launch_k(kern_t, dim3(n_slices * best), dim3(kDecDownThreads), smem, s, true,
+                  static_cast<unsigned>(best), mw, P, static_cast<const uint32_t *>(touch_ws));
+}
+
+size_t dec_touch_ws_bytes(int M, int d_ff) {
+  return (M > 0 && M <= kDecMaxTokens) ? sizeof(uint32_t) * static_cast<size_t>(d_ff / 32 + 1) : 0;
 }
 
 }  // namespace twell

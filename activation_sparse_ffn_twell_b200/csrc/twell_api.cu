@@ -53,6 +53,8 @@ struct Ws {
   size_t sp;         // excess lists of the 2:4 down path (present when d_model is
                      // given and the shape can use it)
   size_t sp_bytes;
+  size_t touch;      // touched-unit bitmap of the decode-size down kernel
+  size_t touch_bytes;
   size_t total;
 };
 
@@ -68,7 +70,9 @@ Ws ws_plan(int M, int d_ff, int tile_w, int ell_w, int cap, int d_model = 0) {
   TwellView v = {};
   v.M = M; v.f = d_ff; v.tw = tile_w; v.E = ell_w; v.T = d_ff / tile_w;
   w.sp_bytes = (d_model > 0 && sp_eligible(v, d_model)) ? sp_ws_bytes(M, d_ff, d_model) : 0;
-  w.total = align256(w.sp + w.sp_bytes);
+  w.touch = align256(w.sp + w.sp_bytes);
+  w.touch_bytes = d_model > 0 ? dec_touch_ws_bytes(M, d_ff) : 0;
+  w.total = align256(w.touch + w.touch_bytes);
   return w;
 }
 
@@ -194,9 +198,11 @@ twell_status spmm_checked(const twell_matrix *a, const uint16_t *W_down, int d_m
   if (mode == TWELL_DOWN_GATHER)
     return from_cuda(launch_spmm_gather(v, W_down, d_model, y, nullptr, pdl_first, s));
   // decode-size batches: the split-K tensor-core kernel streams W_down over every SM
-  if (decode_down_eligible(a->M))
-    return from_cuda(launch_spmm_decode(v, W_down, d_model, y, sms, pdl_first, s));
   const Ws w = ws_plan(a->M, a->d_ff, a->tile_w, a->ell_w, a->ovf_capacity, d_model);
+  if (decode_down_eligible(a->M)) {
+    uint32_t *touch = w.touch_bytes > 0 ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + w.touch) : nullptr;
+    return from_cuda(launch_spmm_decode(v, W_down, d_model, y, touch, sms, pdl_first, s));
+  }
   int32_t *blk = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + w.blk_path);
   const SplitWs sp = split_ptrs(w, ws);
   if (mode == TWELL_DOWN_SPARSE && w.sp_bytes > 0) {

@@ -179,6 +179,12 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *gsrc) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
                : "memory");
 }
+// 16-byte copy that reads `src_bytes` (0 or 16) and fills the rest with zeros.
+__device__ __forceinline__ void cp_async_16_zfill(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_8(void *smem_dst, const void *gsrc) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
                : "memory");
@@ -200,6 +206,13 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
           smem_u32(smem_dst)),
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Ask L2 for [p, p + bytes) (128-byte lines), no registers or completion.
+__device__ __forceinline__ void prefetch_l2_range(const void *p, size_t bytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~static_cast<uintptr_t>(127);
+  const uintptr_t a1 = reinterpret_cast<uintptr_t>(p) + bytes;
+  for (uintptr_t a = a0; a < a1; a += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

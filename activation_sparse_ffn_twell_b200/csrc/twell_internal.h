@@ -195,8 +195,11 @@ cudaError_t launch_twell_transpose(const TwellView &a, const PackTarget &out, fl
 bool decode_up_eligible(int M, int d_ff, int tile_w);
 bool decode_down_eligible(int M);
 cudaError_t launch_up_pack_decode(const UpArgs &a, const PackTarget &t, int num_sms, cudaStream_t s);
+// touch_ws: dec_touch_ws_bytes(M, d_ff) bytes of workspace for the touched-unit
+// bitmap (NULL: always the streaming kernel).
 cudaError_t launch_spmm_decode(const TwellView &v, const uint16_t *w_down, int d, uint16_t *y,
-                               int num_sms, bool pdl, cudaStream_t s);
+                               uint32_t *touch_ws, int num_sms, bool pdl, cudaStream_t s);
+size_t dec_touch_ws_bytes(int M, int d_ff);
 
 // Down path of a 128-token block (the block-path array the down kernels share).
 constexpr int kPathGather = 0;   // CUDA-core gather (k_spmm_gather)

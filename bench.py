@@ -291,6 +291,8 @@ def run_ours(args):
         up_k = ("k_up_pack", "fused up-GEMM + ReLU + TwELL pack, CTA pairs")
     if args.mode == "gather":
         down_k = ("k_spmm_gather", "CUDA-core gather of W_down rows per nonzero")
+    elif dec_down and _decode_touched(M, f):
+        down_k = ("k_spmm_dec_touched", "decode batch: touched W_down rows only, split-K clusters")
     elif dec_down:
         down_k = ("k_spmm_dec", "decode batch: split-K clusters, DSMEM reduction")
     elif args.mode == "sparse" and _sparse_ok(M, f, tw, E):
@@ -331,7 +333,8 @@ def run_ours(args):
                            "useful_flop": rl["useful_flop"],
                            "unavoidable_bytes": rl["unavoidable_bytes"],
                            "touched_w_down_rows": touched, "peaks": peaks["source"]},
-        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d, _sparse_ok(M, f, tw, E)),
+        "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d, _sparse_ok(M, f, tw, E),
+                                                       dec_down and _decode_touched(M, f)),
         "wall_s_timed_region": wall,
     }
     result["clocks"] = clk.summary()
@@ -391,7 +394,24 @@ def _decode_paths(M, f, tw, mode):
     return (M <= 256 and tw <= 128 and f % 128 == 0), (M <= 256 and mode != "gather")
 
 
-def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False):
+def _decode_touched(M, f):
+    """Decode-size batches whose down-projection takes the touched-unit kernel
+    (the library's rule: up to 32 tokens, d_ff <= 65536; TWELL_DECODE_TOUCHED=0
+    turns it off, =all extends it to every decode-size batch)."""
+    import os
+    sel = os.environ.get("TWELL_DECODE_TOUCHED", "")
+    if sel.startswith("0") or f > 65536:
+        return False
+    if not sel.startswith("a"):
+        return M <= 32
+    # every decode-size batch whose stage ring leaves room for the gather's
+    # lag of 4 stages (the library's check, with the largest unit list)
+    np_ = 16 if M <= 16 else (M + 15) // 16 * 16
+    tables = 8 * (f // 32 + 1) + 2 * ((f + 63) // 64) * 64
+    return M <= 256 and (225 * 1024 - 1536 - tables) // (16384 + np_ * 128) > 4
+
+
+def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False, dec_touched=False):
     # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter.
     # spmm in sparse mode, where the 2:4 path applies: k_sp_prep, k_sp_decide,
     # k_spmm_sp and k_spmm_mma, each tensor kernel taking its own token groups.
@@ -399,7 +419,7 @@ def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False):
     # k_block_path too when the split schedule is possible (d_model > 256: it
     # zeroes the arrival counters); the decode-size down path is one kernel.
     if dec_down:
-        return 4 + 1
+        return 4 + (2 if dec_touched else 1)   # k_dec_touch before the touched-unit kernel
     if sparse_ok and mode == "sparse":
         return 4 + 4   # k_sp_prep, k_sp_decide, k_spmm_sp, k_spmm_mma
     if mode == "auto":

@@ -53,7 +53,11 @@ typedef enum {
   TWELL_DOWN_AUTO = 0,   /* per 128-token block, by measured density crossover:
                             GATHER below it, MMA at or above it                   */
   TWELL_DOWN_GATHER = 1, /* CUDA-core gather of W_down rows per packed nonzero    */
-  TWELL_DOWN_MMA = 2,    /* tcgen05 tensor cores on h tiles rebuilt from TwELL    */
+  TWELL_DOWN_MMA = 2,    /* tcgen05 tensor cores on h tiles rebuilt from TwELL.
+                            AUTO and MMA with M <= 256 take the decode-size
+                            split-K kernel (tokens on the MMA's N side); up to
+                            32 tokens it runs on the hidden units some token
+                            uses, reading only their W_down rows                */
   TWELL_DOWN_SPARSE = 3  /* tcgen05 2:4 structured-sparse tensor cores: per group
                             of 4 hidden units the first two nonzeros run on the
                             sparse MMA, the rest are added on CUDA cores.  Taken
@@ -102,7 +106,10 @@ const char *twell_status_string(twell_status s);
  * 0 or 1.  Returns 0 for invalid shapes.  The workspace is scratch: its contents
  * need no initialisation and are undefined after a call.  For M > 256 and
  * d_model > 256 it includes 80 MiB of fp32 partial tiles used when the
- * tensor-core down-projection shares 128 x 512 tiles of y between SMs.
+ * tensor-core down-projection shares 128 x 512 tiles of y between SMs; for
+ * 1 <= M <= 256 it includes a bitmap of d_ff / 32 + 1 words, the hidden units
+ * that some token of the batch uses (the decode-size down-projection of up to
+ * 32 tokens reads only those rows of W_down).
  */
 size_t twell_workspace_bytes(int M, int d_model, int d_ff, int tile_w, int ell_w, int gated,
                              int ovf_capacity);

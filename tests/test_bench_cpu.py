@@ -72,3 +72,4 @@ def test_kernels_per_step():
     assert bench._kernels_per_step("gather", False, 2048) == 5
     # decode-size: the split-K down kernel alone
     assert bench._kernels_per_step("auto", True, 4096) == 5
+    assert bench._kernels_per_step("auto", True, 4096, False, True) == 6   # + k_dec_touch

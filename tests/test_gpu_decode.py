@@ -124,3 +124,97 @@ def test_decode_and_gather_agree_on_the_same_twell():
     y_gat = T.twell_spmm(a, dev(L.w_down), mode="gather")
     assert_y_close(y_mma, y_ref)
     assert_y_close(y_gat, y_ref)
+
+
+# Batches of at most 32 tokens take the touched-unit down kernel: a bitmap of
+# the hidden units some token uses, compacted K, W_down rows gathered for those
+# units only (or every row streamed when more than 3/4 of the units are touched).
+TOUCHED_CASES = [
+    # M, d, f, tw, E, rho
+    (1, 256, 1024, 128, 16, 0.05),     # gather mode; most CTAs of a cluster get no K step
+    (32, 4096, 2048, 128, 8, 0.02),    # gather mode over 32 column slices
+    (2, 128, 4096, 128, 8, 0.20),      # every pair overflows: backup segments read by unit list
+    (4, 128, 2048, 64, 5, 0.10),       # ell_w % 8 != 0: per-slot builder
+    (3, 128, 1024, 32, 4, 0.05),       # tile_w 32
+    (20, 128, 1024, 256, 24, 0.05),    # tile_w 256
+    (17, 64, 512, 64, 8, 0.10),        # more than 3/4 touched: streaming inside the same kernel
+    (32, 192, 1024, 128, 16, 0.01),    # largest batch of the kernel, a ragged column slice
+    (64, 192, 1024, 128, 16, 0.01),    # above it: the streaming kernel
+]
+
+
+@pytest.mark.parametrize("M,d,f,tw,E,rho", TOUCHED_CASES)
+def test_decode_touched_units_spmm(M, d, f, tw, E, rho):
+    L = S.small_random(M, d, f, tw, E, rho, seed=M * 7 + f + tw)
+    h = O.hidden(L.x, L.w_up, L.b, L.w_gate)
+    ref = O.twell_pack(h, tw, E)
+    a = upload_twell(ref, cap=max(ref.n_ovf, 1))
+    y = T.twell_spmm(a, dev(L.w_down), mode="mma")
+    assert T.read_status(a)[0] == 0
+    assert_y_close(y, O.twell_spmm(ref, L.w_down))
+
+
+def test_decode_touched_zero_density_is_exact_zero():
+    """No unit touched: compacted K is empty, every CTA stores a zero partial."""
+    L = S.small_random(32, 512, 1024, 128, 16, 0.0)
+    ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), 128, 16)
+    a = upload_twell(ref, cap=1)
+    y = T.twell_spmm(a, dev(L.w_down), mode="mma")
+    assert T.read_status(a)[0] == 0
+    assert torch.count_nonzero(y.float()).item() == 0
+
+
+def test_decode32_full_shape_integer_forward_bitexact():
+    """The decode-size layer at its full shape (32 tokens, 4096 -> 16384, 2 %) on
+    the integer-exact family: TwELL and every y bit through the touched-unit
+    down kernel (about half of W_down's rows gathered)."""
+    L = S.integer_exact(M=32, d_model=4096, d_ff=16384, tile_w=128, density=0.02, seed=32)
+    ref, y64 = O.ffn_forward(L.x, L.w_up, L.b, L.w_down, L.tile_w, L.ell_w)
+    y, a = T.twell_ffn_forward(dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_down), tile_w=128,
+                               ell_w=L.ell_w, mode="auto", ovf_capacity=max(ref.n_ovf, 1))
+    assert T.read_status(a) == (0, ref.n_ovf)
+    got, _ = twell_to_np(a)
+    assert_twell_equal(got, ref)
+    assert np.array_equal(host_bits(y), O.f64_to_bits(O.bf16_round(y64)))
+
+
+_CHILD = r"""
+import sys, numpy as np
+import activation_sparse_ffn_twell_b200 as T, oracle as O, twell_synth as S
+sys.path.insert(0, 'tests')
+from _gpu_helpers import dev, host_bits, upload_twell
+out = {}
+for i, (M, d, f, tw, E, rho) in enumerate(%r):
+    L = S.small_random(M, d, f, tw, E, rho, seed=i + 3)
+    ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), tw, E)
+    a = upload_twell(ref, cap=max(ref.n_ovf, 1))
+    y = T.twell_spmm(a, dev(L.w_down), mode="mma")
+    assert T.read_status(a)[0] == 0
+    out["y%%d" %% i] = host_bits(y)
+np.savez(sys.argv[1], **out)
+"""
+
+FORCED_CASES = [(32, 256, 2048, 128, 8, 0.02), (128, 512, 2048, 128, 8, 0.005),
+                (256, 256, 1024, 64, 8, 0.002), (8, 128, 1024, 128, 8, 0.05)]
+
+
+@pytest.mark.parametrize("setting", ["0", "all"])
+def test_decode_touched_switch(tmp_path, setting):
+    """TWELL_DECODE_TOUCHED=0 keeps every batch on the streaming kernel, =all
+    sends every decode-size batch whose stage ring allows it (gather mode where
+    few units are touched) through the touched-unit kernel; y is within
+    tolerance of the oracle either way."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = tmp_path / "y.npz"
+    env = dict(os.environ, TWELL_DECODE_TOUCHED=setting, PYTHONPATH=root)
+    subprocess.run([sys.executable, "-c", _CHILD % (FORCED_CASES,), str(out)], cwd=root, env=env,
+                   check=True, timeout=600)
+    got = np.load(out)
+    for i, (M, d, f, tw, E, rho) in enumerate(FORCED_CASES):
+        L = S.small_random(M, d, f, tw, E, rho, seed=i + 3)
+        ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), tw, E)
+        y = torch.from_numpy(got["y%d" % i].view(np.int16)).view(torch.bfloat16)
+        assert_y_close(y, O.twell_spmm(ref, L.w_down))
