@@ -612,6 +612,9 @@ def _e2e(T, L, x, wu, b, wd, a, y, args, dev, stream, world):
 
 
 SWEEP_DENSITIES = (0.20, 0.10, 0.05, 0.02, 0.01)
+# --sweep: the forced gather / MMA paths beside auto, with the low densities
+# where the per-block crossover between them lies
+SWEEP_DENSITIES_FINE = (0.20, 0.10, 0.05, 0.03, 0.02, 0.01, 0.005, 0.0025)
 
 
 def _sweep(T, args, dev, peaks, modes=("auto",)):
@@ -641,7 +644,7 @@ def _sweep(T, args, dev, peaks, modes=("auto",)):
         torch.cuda.synchronize(dev)
         return _median([p.elapsed_time(q) for p, q in evs])
 
-    for rho in SWEEP_DENSITIES:
+    for rho in (SWEEP_DENSITIES_FINE if len(modes) > 1 else SWEEP_DENSITIES):
         L = _workload(rho, args.M, args.seed)
         tb = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
         x, wu, b, wd = tb(L.x), tb(L.w_up), tb(L.b), tb(L.w_down)
@@ -783,7 +786,8 @@ def main():
     ap.add_argument("--mode", default="auto", choices=["auto", "gather", "mma", "sparse"])
     ap.add_argument("--workload", default="relu_15b", choices=WORKLOADS,
                     help="default: the 1.5B-scale layer the headline metric is quoted on")
-    ap.add_argument("--sweep", action="store_true", help="add the 20/10/5/1%% density sweep")
+    ap.add_argument("--sweep", action="store_true",
+                    help="density sweep 20%% .. 0.25%% with the forced gather / MMA paths beside auto")
     ap.add_argument("--token-overflow", action="store_true",
                     help="add the whole-token reading of the backup next to the per-pair one")
     ap.add_argument("--backward", action="store_true",

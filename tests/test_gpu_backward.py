@@ -87,3 +87,24 @@ def test_backward_rejects_unsupported_shapes():
     y, h = T.twell_ffn_forward(x, wu, b, wd, tile_w=128, ell_w=16)
     with pytest.raises(T.TwellError):
         T.twell_ffn_backward(x, wu, wd, h, dev(L.x))
+
+
+def test_backward_gaussian_full_shape_1_5b():
+    """The backward pass at the 1.5B layer's full shape (4096 tokens, 2048 ->
+    8192, 5 %), Gaussian weights and output gradient, through the same split
+    schedules the bench times: every gradient within the y tolerance of the
+    oracle's exact sums over the forward's own hidden activations."""
+    L = S.relu_15b(0.05)
+    rng = np.random.default_rng(15)
+    dy = S.bf16_bits_from_f32(rng.standard_normal((L.M, L.d_model)).astype(np.float32))
+    x, wu, b, wd = dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_down)
+    y, h = T.twell_ffn_forward(x, wu, b, wd, tile_w=L.tile_w, ell_w=L.ell_w)
+    assert T.read_status(h)[0] == 0
+    dX, dWu, db, dWd = T.twell_ffn_backward(x, wu, wd, h, dev(dy))
+    assert T.read_status(h)[0] == 0
+    got, _ = twell_to_np(h)
+    g = O.ffn_backward(L.x, L.w_up, L.b, L.w_down, dy, h=O.twell_unpack(got))
+    for name, t in (("dx", dX), ("dw_up", dWu), ("dw_down", dWd)):
+        assert _rel_l2(t, g[name]) <= 2e-3, name
+    dbg = db.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(dbg - g["db"]) <= 2e-3 * np.linalg.norm(g["db"])
