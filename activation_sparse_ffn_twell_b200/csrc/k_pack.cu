@@ -183,6 +183,66 @@ __global__ void __launch_bounds__(256) k_ovf_scatter(PackTarget p) {
   }
 }
 
+// Batches of at most kSmallScanRows tokens: the backup scan and the scatter in
+// one kernel.  Every CTA loads the per-token overflow counts into shared memory
+// and scans them (one warp, 8 tokens per lane); CTA 0 also writes n_ovf and the
+// capacity status.  Then each warp moves its staged segments as k_ovf_scatter.
+constexpr int kSmallScanRows = 256;
+
+template <int TW>
+__global__ void __launch_bounds__(256) k_ovf_finalize_small(PackTarget p) {
+  __shared__ int prefix_s[kSmallScanRows];
+  griddep_launch_dependents();
+  griddep_wait();   // the producer's counts and staged segments
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    int v[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int r = lane * 8 + j;
+      v[j] = r < p.M ? p.row_ovf[r] : 0;
+      tot += v[j];
+    }
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    int run = incl - tot;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      prefix_s[lane * 8 + j] = run;
+      run += v[j];
+    }
+    if (blockIdx.x == 0 && lane == 31) {
+      *p.n_ovf = incl;
+      if (incl > p.cap) raise_status(p.status, TWELL_ERR_OVERFLOW_CAPACITY);
+    }
+  }
+  __syncthreads();
+  const int warps_per_cta = blockDim.x >> 5;
+  const int staged = min(*p.stage_ctr, p.cap);
+  for (int k = blockIdx.x * warps_per_cta + warp; k < staged; k += gridDim.x * warps_per_cta) {
+    const int pos = p.stage_pos[k];
+    const int r = pos / p.T, t = pos - r * p.T;
+    int before = 0;
+    for (int t0 = 0; t0 < t; t0 += 32) {
+      const int tt = t0 + lane;
+      const bool ov = (tt < t) && (static_cast<int>(p.nnz[static_cast<size_t>(r) * p.T + tt]) > p.E);
+      before += __popc(__ballot_sync(0xFFFFFFFFu, ov));
+    }
+    const int rank = prefix_s[r] + before;
+    if (rank >= p.cap) continue;
+    if (lane == 0) p.ovf_pos[rank] = pos;
+    const uint16_t *src = p.stage_dense + static_cast<size_t>(k) * TW;
+    uint16_t *dst = p.ovf_dense + static_cast<size_t>(rank) * TW;
+    constexpr int kVec = TW / 8;
+    for (int c = lane; c < kVec; c += 32)
+      reinterpret_cast<uint4 *>(dst)[c] = reinterpret_cast<const uint4 *>(src)[c];
+  }
+}
+
 // Per token: its tiles' |h| partial sums and TwELL counts added in a fixed
 // order (each lane strides the tiles, then a fixed butterfly), so the result
 // is the same on every run.
@@ -252,6 +312,17 @@ cudaError_t launch_pack_reset(const PackTarget &t, cudaStream_t s) {
 
 cudaError_t launch_overflow_finalize(const PackTarget &t, cudaStream_t s) {
   if (t.M == 0) return cudaSuccess;
+  if (t.M <= kSmallScanRows) {
+    // one dependent launch: the scan of at most 256 counts is repeated per CTA
+    const dim3 grid(grid_for(t.cap > 0 ? t.cap : 1, 8, 148 * 8)), block(256);
+    switch (t.tw) {
+      case 32: return launch_k(k_ovf_finalize_small<32>, grid, block, 0, s, true, 1, t);
+      case 64: return launch_k(k_ovf_finalize_small<64>, grid, block, 0, s, true, 1, t);
+      case 128: return launch_k(k_ovf_finalize_small<128>, grid, block, 0, s, true, 1, t);
+      case 256: return launch_k(k_ovf_finalize_small<256>, grid, block, 0, s, true, 1, t);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   // both follow the producer kernel of the same call: dependent launches
   cudaError_t e = launch_k(k_ovf_row_scan, dim3(1), dim3(1024), 0, s, true, 1, t);
   if (e != cudaSuccess) return e;

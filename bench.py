@@ -334,7 +334,7 @@ def run_ours(args):
                            "unavoidable_bytes": rl["unavoidable_bytes"],
                            "touched_w_down_rows": touched, "peaks": peaks["source"]},
         "gpu_launches": args.steps * _kernels_per_step(args.mode, dec_down, d, _sparse_ok(M, f, tw, E),
-                                                       dec_down and _decode_touched(M, f)),
+                                                       dec_down and _decode_touched(M, f), M),
         "wall_s_timed_region": wall,
     }
     result["clocks"] = clk.summary()
@@ -411,22 +411,24 @@ def _decode_touched(M, f):
     return M <= 256 and (225 * 1024 - 1536 - tables) // (16384 + np_ * 128) > 4
 
 
-def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False, dec_touched=False):
-    # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter.
+def _kernels_per_step(mode, dec_down=False, d_model=0, sparse_ok=False, dec_touched=False, M=4096):
+    # up_pack: k_pack_reset + the producer + k_ovf_row_scan + k_ovf_scatter (up to
+    # 256 tokens the scan and the scatter are one kernel, k_ovf_finalize_small).
     # spmm in sparse mode, where the 2:4 path applies: k_sp_prep, k_sp_decide,
     # k_spmm_sp and k_spmm_mma, each tensor kernel taking its own token groups.
     # Otherwise auto: k_block_path, gather and k_spmm_mma; mma runs
     # k_block_path too when the split schedule is possible (d_model > 256: it
     # zeroes the arrival counters); the decode-size down path is one kernel.
+    up = 3 if M <= 256 else 4
     if dec_down:
-        return 4 + (2 if dec_touched else 1)   # k_dec_touch before the touched-unit kernel
+        return up + (2 if dec_touched else 1)   # k_dec_touch before the touched-unit kernel
     if sparse_ok and mode == "sparse":
-        return 4 + 4   # k_sp_prep, k_sp_decide, k_spmm_sp, k_spmm_mma
+        return up + 4   # k_sp_prep, k_sp_decide, k_spmm_sp, k_spmm_mma
     if mode == "auto":
-        return 4 + 3
+        return up + 3
     if mode in ("mma", "sparse"):
-        return 4 + (2 if d_model > 256 else 1)
-    return 4 + 1
+        return up + (2 if d_model > 256 else 1)
+    return up + 1
 
 
 def _sparse_ok(M, f, tw, E):

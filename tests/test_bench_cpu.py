@@ -70,6 +70,9 @@ def test_kernels_per_step():
     assert bench._kernels_per_step("mma", False, 2048) == 6
     assert bench._kernels_per_step("mma", False, 256) == 5
     assert bench._kernels_per_step("gather", False, 2048) == 5
-    # decode-size: the split-K down kernel alone
+    # decode-size: the split-K down kernel alone; up to 256 tokens the backup scan
+    # and scatter are one kernel
     assert bench._kernels_per_step("auto", True, 4096) == 5
     assert bench._kernels_per_step("auto", True, 4096, False, True) == 6   # + k_dec_touch
+    assert bench._kernels_per_step("auto", True, 4096, False, False, 128) == 4
+    assert bench._kernels_per_step("auto", True, 4096, False, True, 32) == 5

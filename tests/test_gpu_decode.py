@@ -218,3 +218,24 @@ def test_decode_touched_switch(tmp_path, setting):
         ref = O.twell_pack(O.hidden(L.x, L.w_up, L.b), tw, E)
         y = torch.from_numpy(got["y%d" % i].view(np.int16)).view(torch.bfloat16)
         assert_y_close(y, O.twell_spmm(ref, L.w_down))
+
+
+@pytest.mark.parametrize("M,d,f,tw,E,rho,gated", [
+    (32, 256, 2048, 128, 8, 0.10, False),    # most pairs overflow: units found in backup segments
+    (5, 192, 1024, 64, 8, 0.05, False),
+    (24, 256, 1024, 128, 8, 0.10, True),
+    (1, 128, 512, 128, 16, 0.0, False),      # no unit touched
+])
+def test_fused_decode_forward_touched_units(M, d, f, tw, E, rho, gated):
+    """The fused decode forward up to 32 tokens (backup ordering in one kernel,
+    then the bitmap pass and the touched-unit down kernel): y matches the oracle,
+    including tokens whose hidden units appear only in backup segments, and a
+    separate twell_spmm call on the same TwELL gives the same bits."""
+    L = S.small_random(M, d, f, tw, E, rho, gated=gated, seed=M * 13 + f)
+    y_ref = O.dense_ffn(L.x, L.w_up, L.b, L.w_down, L.w_gate)
+    x, wu, b, wd, wg = dev(L.x), dev(L.w_up), dev(L.b), dev(L.w_down), dev(L.w_gate)
+    y, a = T.twell_ffn_forward(x, wu, b, wd, tile_w=tw, ell_w=E, W_gate=wg, ovf_capacity=M * (f // tw))
+    assert T.read_status(a)[0] == 0
+    assert_y_close(y, y_ref)
+    y2 = T.twell_spmm(a, wd)
+    assert np.array_equal(host_bits(y), host_bits(y2))
