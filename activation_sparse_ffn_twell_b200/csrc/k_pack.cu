@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(1024) k_ovf_row_scan(PackTarget p) {
       run += v[j];
     }
     carry += carry_s;
-    __syncthreads();   // warp_sums / carry_s are rewritten by the next round
+    __syncthreads();   // warp_sums / carry_s are rewritten by the next pass of the loop
   }
   if (tid == 0) {
     *p.n_ovf = carry;
