@@ -947,9 +947,16 @@ void plan_split(DownParams &P, int M, int d, int num_sms) {
         P.grid = tiles * parts;
       }
     } else {
-      // only when the deal is shorter than the whole-tile waves on every SM
+      // only when the deal is shorter than the whole-tile waves on every SM, and
+      // only for tiles of at least kMinDealSteps K steps: a shared tile costs a
+      // partial write and read-back of ~15 us whatever its length.  Measured on
+      // B200: 256 tiles of 64 K steps (the backward's weight-gradient products at
+      // the 1.5B layer) took longer dealt than whole (backward 0.634 against 0.611
+      // ms), 256 tiles of 128 K steps (heavy tail) and 320 of 160 (gated 2B)
+      // took less (down 0.353 against 0.402 ms; 0.377 against 0.423 ms).
+      constexpr int kMinDealSteps = 128;
       const long long waves = (tiles + num_sms - 1) / num_sms;
-      if (tiles % num_sms != 0 && static_cast<long long>(tiles) < waves * g) {
+      if (tiles % num_sms != 0 && static_cast<long long>(tiles) < waves * g && P.num_kb >= kMinDealSteps) {
         P.dp_tiles = 0;
         P.units = static_cast<long long>(tiles) * P.nc;
         long long sk = (P.units * P.ck) / kMinSplitSteps;

@@ -33,6 +33,7 @@ if torch.cuda.is_available():
 
 MIN_SPLIT_STEPS = 32     # K steps per CTA at least
 MAX_SPLIT_CTAS = 160
+MIN_DEAL_STEPS = 128     # K steps per tile for the even deal
 
 
 def _shared_tiles(M, d, f, tw):
@@ -47,7 +48,7 @@ def _shared_tiles(M, d, f, tw):
     if tiles < g:
         parts = min(g // tiles, nc * ck // MIN_SPLIT_STEPS, nc)
         return {t: parts for t in range(tiles)} if parts >= 2 else {}
-    if tiles % g == 0:
+    if tiles % g == 0 or num_kb < MIN_DEAL_STEPS:
         return {}
     U = tiles * nc
     sk = max(1, min(g, U * ck // MIN_SPLIT_STEPS))
@@ -64,7 +65,7 @@ CASES = [
     (520, 640, 4096, 32, 8, 0.10),       # tile_w 32: a chunk is one K step (two hidden tiles)
     (400, 1024, 4096, 256, 24, 0.05),    # tile_w 256: K steps claimed in groups of 3
     (600, 768, 4608, 128, 16, 0.05),     # T = 36 not a multiple of 8: slots fetched per thread
-    (4864, 2048, 3072, 128, 16, 0.05),   # 152 tiles: every tile's chunks dealt over 148 CTAs
+    (4864, 2048, 8192, 128, 16, 0.05),   # 152 tiles of 128 K steps: every tile's chunks dealt over 148 CTAs
 ]
 
 
@@ -85,7 +86,7 @@ def test_split_spmm_against_oracle(M, d, f, tw, E, rho, mode):
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
 
 
-@pytest.mark.parametrize("M,d,f", [(896, 1024, 4096), (4864, 2048, 3072)])
+@pytest.mark.parametrize("M,d,f", [(896, 1024, 4096), (4864, 2048, 8192)])
 def test_split_mixed_paths_auto(M, d, f):
     """AUTO with some 128-token blocks below the gather crossover: the split
     schedules skip the gather-owned tiles and the shared ones still add up."""
@@ -104,7 +105,7 @@ def test_split_mixed_paths_auto(M, d, f):
     assert_y_close(y, y_ref)
 
 
-@pytest.mark.parametrize("M,d,f", [(384, 512, 8192), (4864, 2048, 3072)])
+@pytest.mark.parametrize("M,d,f", [(384, 512, 8192), (4864, 2048, 8192)])
 def test_split_integer_family_bitexact(M, d, f):
     assert _shared_tiles(M, d, f, 128)
     L = S.integer_exact(M=M, d_model=d, d_ff=f, tile_w=128, density=0.05, seed=M + f)

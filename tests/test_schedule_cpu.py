@@ -31,7 +31,8 @@ SHAPES = [
     (700, 768, 4096, 64, 8),         # ragged M and d_model
     (520, 640, 4096, 32, 8),         # tile_w 32
     (400, 1024, 4096, 256, 24),      # tile_w 256
-    (4864, 2048, 3072, 128, 16),     # 152 tiles
+    (4864, 2048, 3072, 128, 16),     # 152 tiles of 48 K steps: whole
+    (8192, 2048, 4096, 128, 16),     # 256 tiles of 64 K steps: whole
     (16384, 4096, 16384, 128, 16),   # 1024 tiles
     (300, 320, 2048, 128, 16),       # few K steps: whole tiles
 ]
@@ -98,6 +99,9 @@ def test_schedule_choice(T):
     s = T.down_schedule(384, 512, 8192, 128, 16, 148)
     assert s["split"] == 1 and s["ctas"] == 12                                 # 3 tiles x 4
     assert T.down_schedule(8192, 2560, 10240, 128, 16, 148)["split"] == 2
+    assert T.down_schedule(8192, 2048, 8192, 128, 24, 148)["split"] == 2        # heavy tail: 128 K steps
+    # 256 tiles of 64 K steps (the backward's weight-gradient products): whole tiles
+    assert T.down_schedule(8192, 2048, 4096, 128, 16, 148)["split"] == 0
     assert T.down_schedule(300, 320, 2048, 128, 16, 148)["split"] == 0          # 32 K steps
     assert T.down_schedule(8192, 2560, 10240, 128, 16, 160)["split"] == 0      # two whole waves
     assert T.down_schedule(21760, 1024, 4096, 128, 16, 200)["split"] == 0      # 340 tiles: deal not shorter
