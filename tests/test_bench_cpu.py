@@ -76,3 +76,16 @@ def test_kernels_per_step():
     assert bench._kernels_per_step("auto", True, 4096, False, True) == 6   # + k_dec_touch
     assert bench._kernels_per_step("auto", True, 4096, False, False, 128) == 4
     assert bench._kernels_per_step("auto", True, 4096, False, True, 32) == 5
+
+
+def test_decode_touched_rule(monkeypatch):
+    """The bench's restatement of the library's choice of the touched-unit decode
+    kernel: up to 32 tokens by default, never with TWELL_DECODE_TOUCHED=0, every
+    decode-size batch whose stage ring allows it with =all."""
+    monkeypatch.delenv("TWELL_DECODE_TOUCHED", raising=False)
+    assert bench._decode_touched(32, 16384) and not bench._decode_touched(33, 16384)
+    assert not bench._decode_touched(32, 131072)            # d_ff above 65536
+    monkeypatch.setenv("TWELL_DECODE_TOUCHED", "0")
+    assert not bench._decode_touched(1, 16384)
+    monkeypatch.setenv("TWELL_DECODE_TOUCHED", "all")
+    assert bench._decode_touched(128, 16384) and not bench._decode_touched(256, 16384)
